@@ -1,0 +1,48 @@
+// common.cuh -- pieces shared by the forward and backward kernels: the device
+// error word and the bounded mbarrier wait.
+#pragma once
+
+#include <cstdint>
+
+#include "sm100.cuh"
+
+namespace fa {
+
+// Device error word of this library (one per device).  A kernel whose bounded
+// wait runs out ORs a code into it; the host reads and clears it in
+// fa_check_device_error.
+__device__ unsigned int g_error_word;
+
+// Codes ORed into the error word: which kernel and which role gave up.
+enum : unsigned int {
+  kErrFwd = 1u << 0,
+  kErrBwdMain = 1u << 1,
+  kErrBwdPre = 1u << 2,
+  kErrRoleLoad = 1u << 8,
+  kErrRoleMma = 1u << 9,
+  kErrRoleSoftmax = 1u << 10,
+  kErrRoleEpilogue = 1u << 11,
+  kErrRoleDrain = 1u << 12,
+  kErrRoleDq = 1u << 13,
+};
+
+// Bounded wait on an mbarrier phase.  Returns true when the phase with the
+// given parity has completed; returns false (after recording `code` in the
+// error word and raising the CTA's abort flag) once `limit_ns` nanoseconds
+// pass, or as soon as another role of the CTA has raised the abort flag.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                             volatile int* abort_flag, unsigned int code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_error_word, code);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,343 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument checks, TMA
+// descriptor encoding, kernel selection and launch, error word, timing.
+//
+// This is the only translation unit of the library: the kernels are included
+// from their headers so that they can all name the one device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/fa.h"
+#include "bwd.cuh"
+#include "fwd.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s per bounded wait
+
+// ------------------------------------------------------------ TMA encoding
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor [BH, rows, cols] (cols innermost), box = 64 cols x box_rows rows
+// x 1, 128-byte swizzle.  Out-of-range loads read zeros; stores are clipped.
+bool encode_bf16_3d(CUtensorMap* map, const void* ptr, int cols, int rows, int bh, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2,
+                           static_cast<cuuint64_t>(cols) * 2 * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// --------------------------------------------------------------- timing
+struct TimedLaunch {
+  int kernel;
+  cudaEvent_t start, stop;
+};
+struct Timing {
+  std::mutex mu;
+  bool active = false;
+  std::vector<TimedLaunch> launches;
+  std::vector<cudaEvent_t> pool;
+} g_timing;
+
+constexpr size_t kMaxTimed = 65536;
+
+cudaEvent_t pool_event() {
+  if (!g_timing.pool.empty()) {
+    cudaEvent_t e = g_timing.pool.back();
+    g_timing.pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets one launch with events when a timing session is open.
+struct LaunchTimer {
+  cudaStream_t stream;
+  int kernel;
+  cudaEvent_t start = nullptr, stop = nullptr;
+  LaunchTimer(cudaStream_t s, int k) : stream(s), kernel(k) {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    if (!g_timing.active || g_timing.launches.size() >= kMaxTimed) return;
+    start = pool_event();
+    stop = pool_event();
+    if (start && stop) cudaEventRecord(start, stream);
+  }
+  ~LaunchTimer() {
+    if (!(start && stop)) return;
+    cudaEventRecord(stop, stream);
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    g_timing.launches.push_back({kernel, start, stop});
+  }
+};
+
+// ------------------------------------------------------------ helpers
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_common(int B, int H, int N, int d, float scale) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > 0x7fffffffLL) return FA_ERR_SHAPE;
+  if (N > (65535 * 128)) return FA_ERR_SHAPE;  // grid.y limit of the Q-tile axis
+  if (static_cast<long long>(N) * bh > (1LL << 40)) return FA_ERR_SHAPE;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
+  if (!std::isfinite(scale)) return FA_ERR_SCALE;
+  return FA_OK;
+}
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct BwdWorkspace {
+  float* dq_acc;  // [BH, Np, d]
+  float* dvec;    // [BH, Np]
+  float* lse2;    // [BH, Np]
+  size_t bytes;
+};
+
+BwdWorkspace bwd_workspace_layout(void* base, int B, int H, int N, int d) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t np = round_up(static_cast<size_t>(N), 128);
+  const size_t acc = bh * np * d * sizeof(float);
+  const size_t vec = round_up(bh * np * sizeof(float), 256);
+  char* p = static_cast<char*>(base);
+  BwdWorkspace w;
+  w.dq_acc = reinterpret_cast<float*>(p);
+  w.dvec = reinterpret_cast<float*>(p + acc);
+  w.lse2 = reinterpret_cast<float*>(p + acc + vec);
+  w.bytes = acc + 2 * vec;
+  return w;
+}
+
+template <int D, bool C>
+fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mo, float* lse, int BH, int N, float scale_log2,
+                     cudaStream_t st) {
+  using L = fa::FwdLayout<D>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return FA_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (!set_smem(fa::fwd_kernel<D, C>, L::kSmemAlloc)) return FA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>((N + L::kBM - 1) / L::kBM));
+  {
+    LaunchTimer timer(st, FA_KERNEL_FWD);
+    fa::fwd_kernel<D, C><<<grid, 256, L::kSmemAlloc, st>>>(mq, mk, mv, mo, lse, N, scale_log2,
+                                                          kWaitLimitNs);
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool C>
+fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mdo, const void* o, const void* dout, const float* lse,
+                     void* dq, void* dk, void* dv, const BwdWorkspace& ws, int BH, int N,
+                     float scale, cudaStream_t st) {
+  using L = fa::BwdLayout<D>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return FA_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (!set_smem(fa::bwd_main_kernel<D, C>, L::kSmemAlloc)) return FA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  const int np = static_cast<int>(round_up(static_cast<size_t>(N), 128));
+  const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  {
+    LaunchTimer timer(st, FA_KERNEL_BWD_PRE);
+    const long long rows = static_cast<long long>(BH) * np;
+    const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);  // 8 rows (warps) per block
+    fa::bwd_preprocess_kernel<D><<<blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
+        ws.dvec, ws.lse2, ws.dq_acc, BH, N, np, static_cast<float>(1.4426950408889634));
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  {
+    LaunchTimer timer(st, FA_KERNEL_BWD_MAIN);
+    dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(np / 128));
+    fa::bwd_main_kernel<D, C><<<grid, L::kThreads, L::kSmemAlloc, st>>>(
+        mq, mk, mv, mdo, ws.dvec, ws.lse2, ws.dq_acc, static_cast<__nv_bfloat16*>(dk),
+        static_cast<__nv_bfloat16*>(dv), N, np, scale, scale_log2, kWaitLimitNs);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  {
+    LaunchTimer timer(st, FA_KERNEL_BWD_DQ);
+    const long long elems = static_cast<long long>(BH) * N * D;
+    const unsigned blocks = static_cast<unsigned>((elems / 8 + 255) / 256);
+    fa::dq_convert_kernel<D><<<blocks, 256, 0, st>>>(ws.dq_acc, static_cast<__nv_bfloat16*>(dq),
+                                                      BH, N, np, scale);
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGN;
+  const int bh = B * H;
+  CUtensorMap mq, mk, mv, mo;
+  if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
+      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mo, o, d, N, bh, 128))
+    return FA_ERR_CUDA;
+  const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return causal ? launch_fwd<64, true>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
+                  : launch_fwd<64, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
+  return causal ? launch_fwd<128, true>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
+                : launch_fwd<128, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.0f) != FA_OK) return 0;
+  return bwd_workspace_layout(nullptr, B, H, N, d).bytes;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, int B, int H, int N, int d, int causal, float scale,
+                 void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGN;
+  const size_t need = bwd_workspace_layout(nullptr, B, H, N, d).bytes;
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGN;
+  const int bh = B * H;
+  BwdWorkspace ws = bwd_workspace_layout(workspace, B, H, N, d);
+  CUtensorMap mq, mk, mv, mdo;
+  if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
+      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mdo, dout, d, N, bh, 128))
+    return FA_ERR_CUDA;
+#ifndef FA_BWD_MAIN_READY
+  return FA_ERR_CUDA;  // backward main kernel not built yet
+#endif
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return causal ? launch_bwd<64, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,
+                                         scale, s)
+                  : launch_bwd<64, false>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,
+                                          scale, s);
+  return causal ? launch_bwd<128, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,
+                                        scale, s)
+                : launch_bwd<128, false>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,
+                                         scale, s);
+}
+
+fa_status fa_check_device_error(void* stream, unsigned int* detail) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, fa::g_error_word, sizeof(word)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (word && cudaMemcpyToSymbol(fa::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (detail) *detail = word;
+  return word ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+}
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL: return "null pointer argument";
+    case FA_ERR_SHAPE: return "invalid shape (B, H, N must be >= 1 and within limits)";
+    case FA_ERR_UNSUPPORTED_D: return "unsupported head dimension (d must be 64 or 128)";
+    case FA_ERR_ALIGN: return "tensor pointer not 16-byte aligned";
+    case FA_ERR_SCALE: return "scale is not finite";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA runtime error";
+    case FA_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case FA_ERR_STATE: return "timing calls out of order";
+  }
+  return "unknown status";
+}
+
+fa_status fa_timing_begin(void) {
+  std::lock_guard<std::mutex> lock(g_timing.mu);
+  if (g_timing.active) return FA_ERR_STATE;
+  g_timing.active = true;
+  return FA_OK;
+}
+
+fa_status fa_timing_end(float* ms_per_kernel, int* launches_per_kernel) {
+  std::vector<TimedLaunch> done;
+  {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    if (!g_timing.active) return FA_ERR_STATE;
+    g_timing.active = false;
+    done.swap(g_timing.launches);
+  }
+  float ms[FA_KERNEL_COUNT] = {0};
+  int cnt[FA_KERNEL_COUNT] = {0};
+  fa_status st = FA_OK;
+  for (auto& l : done) {
+    float t = 0.f;
+    if (cudaEventSynchronize(l.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, l.start, l.stop) != cudaSuccess)
+      st = FA_ERR_CUDA;
+    ms[l.kernel] += t;
+    cnt[l.kernel] += 1;
+  }
+  {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    for (auto& l : done) {
+      g_timing.pool.push_back(l.start);
+      g_timing.pool.push_back(l.stop);
+    }
+  }
+  for (int i = 0; i < FA_KERNEL_COUNT; ++i) {
+    if (ms_per_kernel) ms_per_kernel[i] = ms[i];
+    if (launches_per_kernel) launches_per_kernel[i] = cnt[i];
+  }
+  return st;
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

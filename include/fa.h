@@ -1,0 +1,147 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * The library computes exact scaled-dot-product attention FlashAttention-style:
+ *
+ *   O = softmax(scale * Q K^T) V                        (forward)
+ *   dQ, dK, dV = gradients of sum(dO * O)               (backward)
+ *
+ * Sources for the operations (page title, then section):
+ *   - "FlashAttention为什么更快更省显存" (hi-bin.com lesson 16), opening formula:
+ *     Attention(Q,K,V) = softmax(QK^T / sqrt(d_k)) V; section 把整张表改为分块计算:
+ *     a Q block stays on chip while K/V blocks stream past; section
+ *     反向传播为什么还要重算: the backward recomputes scores from Q, K, V and a
+ *     few saved statistics.
+ *   - "从零实现 FlashAttention-2：分块在线 Softmax", section 在线 softmax：重缩放恒等式:
+ *     running max m and sum l per row, the output accumulator rescaled by
+ *     exp(m_old - m_new), final O = O_final / l_final; section 反向传播：重算，
+ *     而不是存储: the backward keeps only Q, K, V, O and per-row statistics;
+ *     section 提示: the causal mask hides keys whose position is greater than
+ *     the query's, applied inside the tile loop.
+ *   - "FlashAttention 为什么能节省显存并提速,是否改变注意力结果?" (mianstack.com
+ *     q-0277), section 难点在于分块后softmax如何归一: the (m, l, u) merge rule.
+ *
+ * Layout (all calls): Q, K, V, O, dO, dQ, dK, dV are bf16 tensors of shape
+ * [B, H, N, d], row-major and contiguous (d innermost).  LSE is fp32 [B, H, N]:
+ * the natural-log logsumexp of each row of scale * Q K^T over its unmasked
+ * keys.  Query and key sequence lengths are equal (N).  d must be 64 or 128.
+ * Causal masking keeps key j for query i iff j <= i.
+ *
+ * Ownership: the caller owns every buffer (device memory) and the stream.  The
+ * library allocates no device memory, keeps no per-call state, and never
+ * synchronises except inside fa_check_device_error and fa_timing_end.  Calls
+ * are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ * stream).  Concurrent calls on different streams must use distinct output
+ * and workspace buffers.
+ *
+ * Errors: arguments are checked before anything is launched; a failing check
+ * returns its code and launches nothing.  A launch failure returns
+ * FA_ERR_CUDA.  Every wait inside the kernels is bounded: a wait that runs out
+ * makes the kernel record the fact in a device error word and return early;
+ * fa_check_device_error reports it as FA_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef EXACT_ATTENTION_B200_FA_H
+#define EXACT_ATTENTION_B200_FA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_NULL = 1,            /* a required pointer is NULL                      */
+  FA_ERR_SHAPE = 2,           /* B, H or N < 1, or a size overflows              */
+  FA_ERR_UNSUPPORTED_D = 3,   /* d is not 64 or 128                              */
+  FA_ERR_ALIGN = 4,           /* a tensor pointer is not 16-byte aligned         */
+  FA_ERR_SCALE = 5,           /* scale is NaN or infinite                        */
+  FA_ERR_WORKSPACE = 6,       /* workspace NULL or smaller than required         */
+  FA_ERR_CUDA = 7,            /* a CUDA runtime call or launch failed            */
+  FA_ERR_DEVICE_TIMEOUT = 8,  /* a kernel gave up on a bounded wait              */
+  FA_ERR_STATE = 9            /* timing calls out of order                       */
+} fa_status;
+
+/*
+ * Forward pass.
+ *   q, k, v : bf16 [B, H, N, d] device pointers, 16-byte aligned, read only.
+ *   o       : bf16 [B, H, N, d] output, 16-byte aligned.
+ *   lse     : fp32 [B, H, N] output (natural log of the row sum of
+ *             exp(scale * q_i . k_j) over unmasked keys j).
+ *   causal  : 0 = every key, nonzero = keys j <= i only.
+ *   scale   : any finite float (the usual value is 1/sqrt(d)).
+ * Deterministic: the same inputs give bitwise the same outputs.
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator
+ * [B, H, Np, d] plus two fp32 per-row vectors [B, H, Np] (D = rowsum(dO * O)
+ * and the log2-domain LSE), with Np = N rounded up to a multiple of 128.
+ * Returns 0 if the arguments are invalid.
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass (recomputes the score tiles; no N x N tensor is stored).
+ *   q, k, v, o, dout : bf16 [B, H, N, d] device pointers (o from fa_fwd).
+ *   lse              : fp32 [B, H, N] from fa_fwd with the same causal/scale.
+ *   dq, dk, dv       : bf16 [B, H, N, d] outputs.
+ *   workspace        : device scratch of at least fa_bwd_workspace_size bytes,
+ *                      16-byte aligned; its contents on entry do not matter.
+ * dK and dV are written by exactly one CTA per 128-key tile (no atomics); dQ
+ * is summed in fp32 with atomic adds, so it is not bitwise reproducible from
+ * run to run (the rounding order of the adds varies).
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes,
+                 int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT (a bounded wait ran
+ * out; *detail, if non-NULL, receives which one) or FA_ERR_CUDA.
+ */
+FA_API fa_status fa_check_device_error(void* stream, unsigned int* detail);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FA_API const char* fa_status_string(fa_status s);
+
+/* Kernel identifiers for the timing calls below. */
+typedef enum {
+  FA_KERNEL_FWD = 0,       /* forward kernel                         */
+  FA_KERNEL_BWD_PRE = 1,   /* backward: D = rowsum(dO*O), clears dQ  */
+  FA_KERNEL_BWD_MAIN = 2,  /* backward: per-KV-tile main kernel      */
+  FA_KERNEL_BWD_DQ = 3,    /* backward: dQ fp32 -> bf16              */
+  FA_KERNEL_COUNT = 4
+} fa_kernel_id;
+
+/*
+ * Measurement support.  Between fa_timing_begin and fa_timing_end every kernel
+ * this library launches is bracketed by CUDA events recorded on the stream it
+ * is launched on.  fa_timing_end synchronises those events and writes, per
+ * fa_kernel_id, the summed milliseconds and the launch count into the caller's
+ * arrays of FA_KERNEL_COUNT entries (either may be NULL).  Off by default;
+ * at most 65536 launches are recorded per session.  Not thread-safe with
+ * respect to concurrent fa_timing_* calls.
+ */
+FA_API fa_status fa_timing_begin(void);
+FA_API fa_status fa_timing_end(float* ms_per_kernel, int* launches_per_kernel);
+
+/* Library version, major*10000 + minor*100 + patch. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_B200_FA_H */

