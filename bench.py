@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Throughput of the exact-attention training step (causal fwd + bwd) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload c3|c4]
+
+One step = the forward kernel (O, LSE) plus the backward (preprocess, main,
+dQ convert) on one batch of seeded synthetic bf16 inputs that are already
+resident in HBM.  The default workload is B=2, H=16, N=4096, d=128, causal
+(the training-step configuration); the L2 cache is flushed before every timed
+step by writing a 256 MiB buffer outside the step's events.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
+independent (batch, head) problems -- attention has no exchange step across
+heads, so there is no collective on the data path ("scaling": "weak"); the
+step time is the max over ranks.
+
+Metric: algorithmic TFLOP/s, FLOPs = 4*B*H*N^2*d (forward; halved when causal)
+and 2.5 times that for the backward.
+
+``--impl reference`` times the CPU float64 oracle (the reference arm of this
+library: there is no reference GPU code) on a bounded per-step sample of the
+same workload on the host cores, and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd / fwd+bwd TFLOP/s (bf16, causal, d=128) and % of BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def attention_flops(B, H, N, d, causal):
+    fwd = 4.0 * B * H * N * N * d
+    if causal:
+        fwd /= 2.0
+    return fwd, 2.5 * fwd
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest():
+    """Hash of the kernel sources: ncu counters are only valid for this exact code."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_attention_117_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it matches this code."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            data = json.load(f)
+    except Exception:
+        return None
+    ent = data.get(workload, {}).get(kernel_key)
+    if not ent or ent.get("source_digest") != source_digest():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+                parts = [x.strip() for x in out.stdout.strip().split(",")]
+                if len(parts) == 7:
+                    self.samples.append(parts)
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._t.join(timeout=10)
+        return False
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if s[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((x.get("num_threads", 0) for x in info), default=0)
+        return int(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(w, budget_s, device_inputs=None):
+    """Times the float64 oracle (fwd + bwd) on whole (b, h) slices for ~budget_s.
+
+    Returns (algorithmic TFLOP/s, description of the sample).
+    """
+    import numpy as np
+    import torch
+
+    import oracle
+    from exact_attention_117_b200.workloads import make_inputs, sample_slices
+
+    if device_inputs is None:
+        device_inputs = make_inputs(w, "cpu")
+    causal = True
+    fwd1, bwd1 = attention_flops(1, 1, w.N, w.d, causal)
+    order = sample_slices(w.B * w.H, w.B * w.H)
+    done, t_total = 0, 0.0
+    for idx in order:
+        b, h = idx // w.H, idx % w.H
+        sl = [device_inputs[k][b, h].float().cpu().numpy().astype(np.float64)
+              for k in ("q", "k", "v", "do")]
+        t0 = time.perf_counter()
+        oracle.attention_forward(sl[0], sl[1], sl[2], causal=causal, scale=w.scale)
+        oracle.attention_backward(*sl, causal=causal, scale=w.scale)
+        t_total += time.perf_counter() - t0
+        done += 1
+        if t_total >= budget_s:
+            break
+    del torch
+    tflops = done * (fwd1 + bwd1) / t_total / 1e12
+    return tflops, (f"{done} of {w.B * w.H} (b,h) slices of the workload, fwd+bwd in float64 "
+                    f"({t_total:.1f} s)")
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    from exact_attention_117_b200.workloads import make_inputs
+    x = make_inputs(w, "cpu")
+    budget = max(0.5, min(10.0, 150.0 / max(1, steps + warm)))
+    for _ in range(warm):
+        oracle_sample(w, budget * 0.25, x)
+    vals, descs = [], []
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        v, d = oracle_sample(w, budget, x)
+        vals.append(v)
+        descs.append(d)
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+        "ms_per_step": 1000.0 * wall / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True,
+                   "sample": "bounded per-step sample of (b,h) slices"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
+                         "kind": "oracle", "sample": descs[-1]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from exact_attention_117_b200 import fa
+    from exact_attention_117_b200.workloads import make_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    fa.load()
+    causal = True
+    B, H, N, d = w.B, w.H, w.N, w.d
+    fwd_f, bwd_f = attention_flops(B, H, N, d, causal)
+    x = make_inputs(w, dev)
+    q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(fa.workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.forward(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream)
+        fa.backward(q, k, v, o, lse, do, causal=causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                    workspace=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    fa.check_device_error(stream)
+
+    # ---------------------------------------------------------- device-timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    evf = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk, fa.KernelTimer() as kt:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            evf[i][0].record(stream)
+            fa.forward(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse, stream=stream)
+            evf[i][1].record(stream)
+            fa.backward(q, k, v, o, lse, do, causal=causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
+                        workspace=ws, stream=stream)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    fa.check_device_error(stream)
+    step_ms = sum(a.elapsed_time(b) for a, b in ev)
+    fwd_ms = sum(a.elapsed_time(b) for a, b in evf)
+    t = torch.tensor([step_ms, fwd_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, fwd_ms = float(t[0]), float(t[1])
+    ms_per_step = step_ms / args.steps
+    fwd_ms_per = fwd_ms / args.steps
+    bwd_ms_per = ms_per_step - fwd_ms_per
+    value = world * (fwd_f + bwd_f) / (ms_per_step * 1e-3) / 1e12
+
+    # ------------------------------------------------------------- end to end
+    e2e = None
+    if not args.no_e2e:
+        host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+        outs_host = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                     for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+        dev_in = {n: torch.empty_like(t) for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+
+        def e2e_step():
+            for n in dev_in:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            fa.forward(dev_in["q"], dev_in["k"], dev_in["v"], causal=causal, scale=w.scale,
+                       out=o, lse=lse, stream=stream)
+            fa.backward(dev_in["q"], dev_in["k"], dev_in["v"], o, lse, dev_in["do"],
+                        causal=causal, scale=w.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
+                        stream=stream)
+            for n, src in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+                outs_host[n].copy_(src, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te[0]) / args.steps
+        e2e = {"value": world * (fwd_f + bwd_f) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": "pinned host -> device copy, fa_fwd + fa_bwd through the C ABI, "
+                       "outputs copied back to pinned host"}
+
+    if rank != 0:
+        return
+
+    # ------------------------------------------------------------------ roofline
+    peaks, peak_src = load_peaks()
+    per_kernel = {kname: (kt.ms[kname] / kt.launches[kname] if kt.launches[kname] else 0.0)
+                  for kname in fa.KERNELS}
+    totals = {kname: kt.ms[kname] for kname in fa.KERNELS}
+    dom = max(totals, key=totals.get)
+    kernel_flops = {"fwd": fwd_f, "bwd_main": bwd_f}
+    peak_tf = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    if dom in kernel_flops:
+        achieved = kernel_flops[dom] / (per_kernel[dom] * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": achieved / peak_tf,
+                "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)"
+                if peak_src == "measured" else "fallback 1590 TFLOP/s",
+                "traffic": ncu_traffic(dom, w.name),
+                "avg_launch_ms": per_kernel[dom],
+                "algorithmic_flops_per_launch": kernel_flops[dom]}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks.get("hbm_gbs"),
+                "unit": "GB/s", "frac": None, "traffic": None}
+    fwd_tf = fwd_f / (per_kernel["fwd"] * 1e-3) / 1e12 if per_kernel["fwd"] else None
+    bwd_tf = bwd_f / (bwd_ms_per * 1e-3) / 1e12
+    kernels = {kname: {"launches": kt.launches[kname], "total_ms": kt.ms[kname],
+                       "share": kt.ms[kname] / max(1e-9, sum(totals.values()))}
+               for kname in fa.KERNELS}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tf, desc = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": desc}
+
+    launches = sum(kt.launches.values())
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: causal fwd+bwd, B={B} H={H} N={N} d={d}",
+                   "B": B, "H": H, "N": N, "d": d, "causal": True, "scale": w.scale,
+                   "per_rank": "independent copy of the batch on every rank",
+                   "l2": "flushed (256 MiB write) before every timed step, outside its events"},
+        "fwd": {"ms": fwd_ms_per, "tflops": fwd_f / (fwd_ms_per * 1e-3) / 1e12,
+                "kernel_tflops": fwd_tf, "pct_of_peak": 100.0 * (fwd_tf or 0) / peak_tf},
+        "bwd": {"ms": bwd_ms_per, "tflops": bwd_tf, "pct_of_peak": 100.0 * bwd_tf / peak_tf},
+        "pct_of_peak": 100.0 * value / world / peak_tf,
+        "roofline": roof,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c3", choices=["c3", "c4"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+
+    from exact_attention_117_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -45,4 +45,16 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
   }
 }
 
+// Wait that ignores the abort flag: used only to let copies already in flight
+// land before the CTA releases its shared memory.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_error_word, kErrRoleDrain);
+      return;
+    }
+  }
+}
+
 }  // namespace fa

@@ -256,9 +256,6 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
       !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mdo, dout, d, N, bh, 128))
     return FA_ERR_CUDA;
-#ifndef FA_BWD_MAIN_READY
-  return FA_ERR_CUDA;  // backward main kernel not built yet
-#endif
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
     return causal ? launch_bwd<64, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,

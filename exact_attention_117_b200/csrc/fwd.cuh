@@ -66,18 +66,6 @@ struct FwdLayout {
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 };
 
-// Wait that ignores the abort flag: used only to let copies already in flight
-// land before the CTA releases its shared memory.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > limit_ns) {
-      atomicOr(&g_error_word, kErrRoleDrain);
-      return;
-    }
-  }
-}
-
 template <int D, bool kCausal>
 __global__ void __launch_bounds__(256, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,

@@ -96,9 +96,18 @@ def attention_forward(q, k, v, causal: bool = False, scale: float | None = None,
 
 
 def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = None,
-                       row_chunk: int = 1024):
-    """Return ``(dQ, dK, dV)`` of ``L = sum(dO * O)`` for one slice (float64)."""
+                       row_chunk: int = 1024, o_for_d=None):
+    """Return ``(dQ, dK, dV)`` of ``L = sum(dO * O)`` for one slice (float64).
+
+    ``D_i`` is ``sum_j P_ij dP_ij`` by default.  If ``o_for_d`` is given, ``D_i``
+    is formed as ``sum_c dO_ic O_ic`` from that O instead -- the same number
+    when ``o_for_d`` is the exact output (``sum_j P_ij dO_i.v_j = dO_i.O_i``);
+    passing a rounded O measures how much the rounding of the stored output
+    alone moves the gradients.
+    """
     q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    if o_for_d is not None:
+        o_for_d = _as_f64(o_for_d)
     n, d = q.shape
     if scale is None:
         scale = default_scale(d)
@@ -111,7 +120,10 @@ def attention_backward(q, k, v, do, causal: bool = False, scale: float | None = 
         dov = do[r0:r1]
         dv += p.T @ dov                      # dV = P^T dO
         dp = dov @ v.T                       # dP = dO V^T
-        dsum = np.sum(p * dp, axis=1, keepdims=True)   # D_i = sum_j P_ij dP_ij
+        if o_for_d is None:
+            dsum = np.sum(p * dp, axis=1, keepdims=True)   # D_i = sum_j P_ij dP_ij
+        else:
+            dsum = np.sum(dov * o_for_d[r0:r1], axis=1, keepdims=True)
         ds = p * (dp - dsum)                 # dS = P o (dP - D)
         dq[r0:r1] = scale * (ds @ k)         # dQ = scale dS K
         dk += scale * (ds.T @ q[r0:r1])      # dK = scale dS^T Q

@@ -56,10 +56,27 @@ def check_lse(lse_gpu: np.ndarray, lse_ref: np.ndarray, what: str = "LSE"):
     return mx
 
 
-def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str):
+def check_grad(g_gpu: np.ndarray, g_ref: np.ndarray, what: str, floor: float = 0.0):
+    """rel-L2 <= 1e-2, plus ``floor`` where a derived rounding floor applies."""
     rl2 = rel_l2(g_gpu, g_ref)
-    assert rl2 <= GRAD_REL_L2, f"{what}: rel-L2 {rl2:.3e} > {GRAD_REL_L2}"
+    tol = GRAD_REL_L2 + floor
+    assert rl2 <= tol, f"{what}: rel-L2 {rl2:.3e} > {tol:.3e} (floor {floor:.3e})"
     return rl2
+
+
+def output_rounding_floor(q, k, v, do, b, h, causal, scale, grads_ref):
+    """rel-L2 by which rounding O to bf16 alone moves each exact gradient.
+
+    The backward forms D_i = sum_c dO_ic O_ic from the stored bf16 O.  At very
+    short rows dQ and dK are differences of a few nearly equal terms and this
+    rounding dominates; it is a property of the bf16 output, not of the
+    kernels.  Returned as (fq, fk, fv); fv is 0 because dV does not use D.
+    """
+    o_ref, _ = oracle_fwd_slice(q, k, v, b, h, causal, scale)
+    pert = oracle.attention_backward(slice_np(q, b, h), slice_np(k, b, h), slice_np(v, b, h),
+                                     slice_np(do, b, h), causal=causal, scale=scale,
+                                     o_for_d=bf16_round(o_ref))
+    return tuple(rel_l2(p, r) for p, r in zip(pert, grads_ref))
 
 
 def slice_np(t: torch.Tensor, b: int, h: int) -> np.ndarray:

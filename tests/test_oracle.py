@@ -271,3 +271,19 @@ def test_matches_torch_cpu_float64(causal):
     assert np.max(np.abs(dq - tq.grad.numpy())) < 1e-12
     assert np.max(np.abs(dk - tk.grad.numpy())) < 1e-12
     assert np.max(np.abs(dv - tv.grad.numpy())) < 1e-12
+
+
+def test_d_from_output_identity():
+    """sum_j P_ij dP_ij equals sum_c dO_ic O_ic, so forming D from the exact O changes nothing."""
+    rng = np.random.default_rng(12)
+    q, k, v, do = (_rand(rng, 23, 6) for _ in range(4))
+    for causal in (False, True):
+        o, _ = attention_forward(q, k, v, causal)
+        a = attention_backward(q, k, v, do, causal)
+        b = attention_backward(q, k, v, do, causal, o_for_d=o)
+        for x, y in zip(a, b):
+            assert np.max(np.abs(x - y)) < 1e-12
+        # a perturbed O moves dQ and dK but never dV (dV does not involve D)
+        c = attention_backward(q, k, v, do, causal, o_for_d=o + 1e-3)
+        assert np.array_equal(c[2], a[2])
+        assert np.max(np.abs(c[0] - a[0])) > 1e-6
