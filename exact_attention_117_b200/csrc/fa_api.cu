@@ -268,6 +268,57 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                                          scale, s);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch of fa_bwd_noalloc: one fixed device array per GPU, never allocated
+// at call time.  Host code only ever sees its address through
+// cudaGetSymbolAddress; the symbol itself is a host-side stand-in.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once
+// per device); nullptr if the lookup fails.
+void* noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, int causal, float scale, void* stream) {
+  // same checks as fa_bwd, in the same order, before the scratch is touched
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGN;
+  const size_t need = bwd_workspace_layout(nullptr, B, H, N, d).bytes;
+  if (need > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_address();
+  if (!scratch) return FA_ERR_CUDA;
+  // the preprocess kernel rewrites every scratch word the main kernel reads
+  // (the fp32 dQ accumulator is cleared, D and the log2 LSE are written)
+  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, H,
+                N, d, causal, scale, stream);
+}
+
 fa_status fa_check_device_error(void* stream, unsigned int* detail) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   unsigned int word = 0, zero = 0;

@@ -52,6 +52,8 @@ def load() -> ctypes.CDLL:
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd.restype = i
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, vp]
+    lib.fa_bwd_noalloc.restype = i
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
     lib.fa_check_device_error.restype = i
     lib.fa_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
     lib.fa_status_string.restype = ctypes.c_char_p
@@ -143,6 +145,38 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] =
     _check(bwd_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
                    _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
                    B, H, N, d, causal, scale, _stream_ptr(stream)), "fa_bwd")
+    return dq, dk, dv
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # FA_BWD_NOALLOC_SCRATCH_BYTES in include/fa.h
+
+
+def bwd_noalloc_raw(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d, causal, scale,
+                    stream) -> int:
+    """Direct call of ``fa_bwd_noalloc`` with raw pointers; returns the status code."""
+    return load().fa_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, B, H, N, d,
+                                 int(bool(causal)), float(scale), stream)
+
+
+def backward_noalloc(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None,
+                     dq=None, dk=None, dv=None, stream=None):
+    """Like ``backward`` but through ``fa_bwd_noalloc``: the library's own fixed
+    scratch array replaces the workspace, so the C call allocates nothing.
+    Problems needing more than ``NOALLOC_SCRATCH_BYTES`` of scratch raise
+    FaError(FA_ERR_WORKSPACE).  (The outputs are allocated here by torch only if
+    the caller does not pass them.)"""
+    _check_qkv(q, k, v, o, do)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be a contiguous fp32 [B, H, N] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    _check(bwd_noalloc_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq),
+                           _ptr(dk), _ptr(dv), B, H, N, d, causal, scale, _stream_ptr(stream)),
+           "fa_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -107,6 +107,42 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * Backward pass that allocates nothing.  (The pages have no counterpart to
+ * this entry point: it exists only for callers that cannot allocate.)
+ *
+ * Same arguments and results as fa_bwd, minus the workspace: the scratch the
+ * backward needs lives in one fixed array of FA_BWD_NOALLOC_SCRATCH_BYTES
+ * bytes of device memory that is part of this library, so the call itself
+ * never calls cudaMalloc or any other allocating routine.  Meant for callers
+ * that may not allocate device memory on the call path: code running under a
+ * host framework that owns all device memory through its own pool (a direct
+ * allocation would bypass it or fail), and latency-critical loops that must
+ * not allocate or free after start-up because cudaFree can synchronise the
+ * device.
+ *
+ * Limits and caveats:
+ *   - A problem needing more than FA_BWD_NOALLOC_SCRATCH_BYTES of scratch
+ *     (the size fa_bwd_workspace_size reports) is rejected with
+ *     FA_ERR_WORKSPACE before anything is launched.
+ *   - Every GPU that loads this library holds the array (32 MiB) until the
+ *     process exits.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array.  Calls whose kernels overlap
+ *     on the GPU (different streams, no ordering between them) race on it;
+ *     order them, e.g. by issuing them on one stream.  Each call rewrites
+ *     every part of the array it reads, so leftovers of an earlier call never
+ *     leak into its result.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout,
+                                void* dq, void* dk, void* dv,
+                                int B, int H, int N, int d, int causal, float scale,
+                                void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT (a bounded wait ran
  * out; *detail, if non-NULL, receives which one) or FA_ERR_CUDA.
