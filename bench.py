@@ -42,6 +42,32 @@ METRIC = "attention fwd / fwd+bwd TFLOP/s (bf16, causal, d=128) and % of BF16 te
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def rank_workload(w, rank):
+    """The batch rank ``rank`` processes: same shapes, its own seeds.
+
+    Attention over different (batch, head) slices shares nothing, so under
+    torchrun every rank runs an independent batch (weak scaling) and no data
+    crosses GPUs.
+    """
+    import dataclasses
+    return dataclasses.replace(w, seed_base=w.seed_base + 1000 * rank)
+
+
+def max_over_ranks(values, world, device=None):
+    """Element-wise max of a list of floats over all ranks (max-over-ranks timing)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_tflops(flops_per_rank_step, world, ms_per_step):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def attention_flops(B, H, N, d, causal):
     fwd = 4.0 * B * H * N * N * d
     if causal:
@@ -222,7 +248,7 @@ def run_ours(args, w, rank, world, local_rank):
     causal = True
     B, H, N, d = w.B, w.H, w.N, w.d
     fwd_f, bwd_f = attention_flops(B, H, N, d, causal)
-    x = make_inputs(w, dev)
+    x = make_inputs(rank_workload(w, rank), dev)
     q, k, v, do = x["q"], x["k"], x["v"], x["do"]
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -267,14 +293,11 @@ def run_ours(args, w, rank, world, local_rank):
     fa.check_device_error(stream)
     step_ms = sum(a.elapsed_time(b) for a, b in ev)
     fwd_ms = sum(a.elapsed_time(b) for a, b in evf)
-    t = torch.tensor([step_ms, fwd_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, fwd_ms = float(t[0]), float(t[1])
+    step_ms, fwd_ms = max_over_ranks([step_ms, fwd_ms], world, dev)
     ms_per_step = step_ms / args.steps
     fwd_ms_per = fwd_ms / args.steps
     bwd_ms_per = ms_per_step - fwd_ms_per
-    value = world * (fwd_f + bwd_f) / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(fwd_f + bwd_f, world, ms_per_step)
 
     # ------------------------------------------------------------- end to end
     e2e = None
@@ -308,11 +331,8 @@ def run_ours(args, w, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te[0]) / args.steps
-        e2e = {"value": world * (fwd_f + bwd_f) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0] / args.steps
+        e2e = {"value": job_tflops(fwd_f + bwd_f, world, e2e_ms), "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "path": "pinned host -> device copy, fa_fwd + fa_bwd through the C ABI, "
                        "outputs copied back to pinned host"}
