@@ -24,6 +24,7 @@ enum : unsigned int {
   kErrRoleEpilogue = 1u << 11,
   kErrRoleDrain = 1u << 12,
   kErrRoleDq = 1u << 13,
+  kErrAlign = 1u << 14,  // dynamic shared memory base not 1 KiB aligned
 };
 
 // Bounded wait on an mbarrier phase.  Returns true when the phase with the
@@ -43,6 +44,17 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
       return false;
     }
   }
+}
+
+// Bounded wait taken by a whole warp whose lanes then issue warp-collective
+// tcgen05.ld / tcgen05.st: all lanes get the same answer (if any lane gave up,
+// every lane reports failure), so those instructions are never executed by
+// part of a warp.
+__device__ __forceinline__ bool wait_bounded_warp(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns, volatile int* abort_flag,
+                                                  unsigned int code) {
+  const bool ok = wait_bounded(bar, parity, limit_ns, abort_flag, code);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Wait that ignores the abort flag: used only to let copies already in flight

@@ -106,7 +106,7 @@ fa_status check_common(int B, int H, int N, int d, float scale) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > 0x7fffffffLL) return FA_ERR_SHAPE;
-  if (N > (65535 * 128)) return FA_ERR_SHAPE;  // grid.y limit of the Q-tile axis
+  if (N > (65535 * 128)) return FA_ERR_SHAPE;  // grid.y limit of the tile axis
   if (static_cast<long long>(N) * bh > (1LL << 40)) return FA_ERR_SHAPE;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
   if (!std::isfinite(scale)) return FA_ERR_SCALE;
@@ -154,10 +154,11 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     if (!set_smem(fa::fwd_kernel<D, C>, L::kSmemAlloc)) return FA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>((N + L::kBM - 1) / L::kBM));
+  const int q_tiles = (N + L::kBM - 1) / L::kBM;
+  dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>((q_tiles + 1) / 2));  // 2 Q tiles per CTA
   {
     LaunchTimer timer(st, FA_KERNEL_FWD);
-    fa::fwd_kernel<D, C><<<grid, 256, L::kSmemAlloc, st>>>(mq, mk, mv, mo, lse, N, scale_log2,
+    fa::fwd_kernel<D, C><<<grid, 384, L::kSmemAlloc, st>>>(mq, mk, mv, mo, lse, N, scale_log2,
                                                           kWaitLimitNs);
   }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -165,9 +166,9 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 
 template <int D, bool C>
 fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& mdo, const void* o, const void* dout, const float* lse,
-                     void* dq, void* dk, void* dv, const BwdWorkspace& ws, int BH, int N,
-                     float scale, cudaStream_t st) {
+                     const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
+                     const void* o, const void* dout, const float* lse, void* dq,
+                     const BwdWorkspace& ws, int BH, int N, float scale, cudaStream_t st) {
   using L = fa::BwdLayout<D>;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
@@ -191,8 +192,8 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     LaunchTimer timer(st, FA_KERNEL_BWD_MAIN);
     dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(np / 128));
     fa::bwd_main_kernel<D, C><<<grid, L::kThreads, L::kSmemAlloc, st>>>(
-        mq, mk, mv, mdo, ws.dvec, ws.lse2, ws.dq_acc, static_cast<__nv_bfloat16*>(dk),
-        static_cast<__nv_bfloat16*>(dv), N, np, scale, scale_log2, kWaitLimitNs);
+        mq, mk, mv, mdo, mdk, mdv, ws.dvec, ws.lse2, ws.dq_acc, N, np, scale, scale_log2,
+        kWaitLimitNs);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   {
@@ -252,19 +253,20 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!aligned16(workspace)) return FA_ERR_ALIGN;
   const int bh = B * H;
   BwdWorkspace ws = bwd_workspace_layout(workspace, B, H, N, d);
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
   if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
-      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mdo, dout, d, N, bh, 128))
+      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mdo, dout, d, N, bh, 128) ||
+      !encode_bf16_3d(&mdk, dk, d, N, bh, 128) || !encode_bf16_3d(&mdv, dv, d, N, bh, 128))
     return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
-    return causal ? launch_bwd<64, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,
+    return causal ? launch_bwd<64, true>(mq, mk, mv, mdo, mdk, mdv, o, dout, lse, dq, ws, bh, N,
                                          scale, s)
-                  : launch_bwd<64, false>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,
+                  : launch_bwd<64, false>(mq, mk, mv, mdo, mdk, mdv, o, dout, lse, dq, ws, bh, N,
                                           scale, s);
-  return causal ? launch_bwd<128, true>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,
+  return causal ? launch_bwd<128, true>(mq, mk, mv, mdo, mdk, mdv, o, dout, lse, dq, ws, bh, N,
                                         scale, s)
-                : launch_bwd<128, false>(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, ws, bh, N,
+                : launch_bwd<128, false>(mq, mk, mv, mdo, mdk, mdv, o, dout, lse, dq, ws, bh, N,
                                          scale, s);
 }
 

@@ -3,27 +3,42 @@
 // Algorithm (page "从零实现 FlashAttention-2：分块在线 Softmax", sections
 // 在线 softmax：重缩放恒等式 and 从 FlashAttention-1 到 FlashAttention-2; page
 // "FlashAttention 为什么能节省显存并提速,是否改变注意力结果?", section
-// 难点在于分块后softmax如何归一): one CTA owns one 128-row Q tile of one
-// (batch, head).  The Q tile stays in shared memory; 128-key K/V tiles stream
-// through a TMA ring; per key tile the CTA computes S = Q K^T on the tensor
-// cores into TMEM, updates the running row max m and sum l, rescales the
-// output accumulator by exp(m_old - m_new) when the max moved (the factor is
-// exactly 1 otherwise: page 2, section 提示), and accumulates O += P V on the
-// tensor cores.  O / l and the row logsumexp are written once at the end; no
+// 难点在于分块后softmax如何归一): Q tiles stay on chip while 128-key K/V
+// tiles stream past; per key tile the running row max m and sum l are updated,
+// the output accumulator is rescaled by exp(m_old - m_new), and O += P V
+// accumulates; O / l and the row logsumexp are written once at the end.  No
 // N x N tensor ever reaches global memory.
 //
-// Causal masking (page 2, section 提示): key tiles wholly above the diagonal
-// are never loaded; the diagonal tile masks key > query inside the tile.
+// One CTA owns TWO consecutive 128-row Q tiles of one (batch, head) and runs
+// them ping-pong: while the softmax warps of one tile work on its scores, the
+// tensor core computes P V and the next S = Q K^T of the other tile.
 //
-// Warp roles (256 threads):
-//   warp 0     : TMA producer (Q once, then K_j / V_j into a kStages ring)
-//   warp 1     : TMEM allocator and tcgen05.mma issuer
-//   warps 2-3  : idle
-//   warps 4-7  : softmax / rescale / epilogue, one thread per query row
-//                (TMEM lane = row, so the row max and row sum stay inside one
-//                thread and need no cross-lane reduction)
+// Warp roles (384 threads):
+//   warp 0      : TMA producer (both Q tiles once, then K_j / V_j rings)
+//   warp 1      : TMEM allocator and tcgen05.mma issuer
+//   warps 2-3   : idle
+//   warps 4-7   : softmax of Q tile 0, one thread per query row
+//   warps 8-11  : softmax of Q tile 1
+// (TMEM lane = row, so a row's max and sum stay inside one thread.)
 //
-// TMEM columns: S double buffer at [0,128) and [128,256), O at [256, 256+D).
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// The bf16 probabilities P_t are written over the first 64 columns of S_t and
+// fed to the P V product as the TMEM A operand.  tcgen05.mma ops from one
+// thread run in issue order, so S_t(j+1) may be issued right after the P V
+// product that reads P_t(j) from the same columns.  A tcgen05.commit arrives
+// only when every earlier MMA of the issuing thread is complete, so when a
+// softmax warp sees S_t(j) ready, P_t(j-1) V is done and O_t is current.
+//
+// Rescaling (page 2, section 提示: the factor is exactly 1 when the max is
+// unchanged): a row keeps its running max until a tile raises it by more than
+// 8 (base-2 units); until then the new probabilities are taken against the
+// old max (they are at most 2^8) and O needs no correction.  O and l always
+// refer to the same max, so O / l and m + log2 l are unchanged in exact
+// arithmetic.  The rescale of O in TMEM is done only when some row of the
+// warp moved its max.
+//
+// Causal masking (page 2, section 提示): key tiles wholly above a Q tile's
+// diagonal are never computed for it; the diagonal tile masks key > query.
 // All exponentials are base 2 with scale*log2(e) folded in; the stored LSE is
 // converted back to natural log.
 #pragma once
@@ -34,16 +49,15 @@ namespace fa {
 
 template <int D>
 struct FwdLayout {
-  static constexpr int kBM = 128;                    // query rows per tile
-  static constexpr int kBN = 128;                    // keys per tile
-  static constexpr int kStages = (D == 64) ? 3 : 2;  // K/V ring depth
+  static constexpr int kBM = 128;                    // query rows per Q tile
+  static constexpr int kBN = 128;                    // keys per K/V tile
+  static constexpr int kStages = (D == 64) ? 4 : 2;  // K and V ring depth
   static constexpr int kTile = kBM * D * 2;          // bytes of a Q, K or V tile
-  static constexpr int kPTile = kBM * kBN * 2;       // bytes of the bf16 P tile
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kTile;
+  static constexpr int kOffQ0 = 0;
+  static constexpr int kOffQ1 = kTile;
+  static constexpr int kOffK = 2 * kTile;
   static constexpr int kOffV = kOffK + kStages * kTile;
-  static constexpr int kOffP = kOffV + kStages * kTile;
-  static constexpr int kOffBar = kOffP + kPTile;
+  static constexpr int kOffBar = kOffV + kStages * kTile;
   static constexpr int kBarArea = 256;
   static constexpr int kBytes = kOffBar + kBarArea;
   static constexpr int kSmemAlloc = kBytes + 1024;  // slack to align the base to 1 KiB
@@ -53,21 +67,27 @@ struct FwdLayout {
   static constexpr int kKEmpty = kKFull + kStages;
   static constexpr int kVFull = kKEmpty + kStages;
   static constexpr int kVEmpty = kVFull + kStages;
-  static constexpr int kSFull = kVEmpty + kStages;  // 2
-  static constexpr int kSFree = kSFull + 2;         // 2
-  static constexpr int kPFull = kSFree + 2;
-  static constexpr int kODone = kPFull + 1;
-  static constexpr int kDrain = kODone + 1;
+  static constexpr int kSFull = kVEmpty + kStages;  // [2]
+  static constexpr int kPFull = kSFull + 2;         // [2]
+  static constexpr int kOFinal = kPFull + 2;        // [2]
+  static constexpr int kDrain = kOFinal + 2;
   static constexpr int kNumBars = kDrain + 1;
   static constexpr int kOffSlot = kOffBar + 8 * kNumBars;  // TMEM base address
   static constexpr int kOffAbort = kOffSlot + 4;
   static_assert(kOffAbort + 4 <= kOffBar + kBarArea, "barrier area too small");
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128;
+  static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
+  static constexpr float kRescaleThreshold = 8.0f;  // base-2 units
+  static constexpr uint32_t kLaunchRegs = 168;      // 65536 / 384, rounded down to 8
+  static constexpr uint32_t kRegsOther = 80;
+  static constexpr uint32_t kRegsSoftmax = 200;
+  static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= 384 * kLaunchRegs, "register split");
 };
 
 template <int D, bool kCausal>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                float* __restrict__ lse_out, int n, float scale_log2, uint64_t limit_ns) {
@@ -86,25 +106,16 @@ __global__ void __launch_bounds__(256, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
-  const int qt = static_cast<int>(gridDim.y) - 1 - static_cast<int>(blockIdx.y);  // heavy first
-  const int n_kv = kCausal ? (qt + 1) : (n + L::kBN - 1) / L::kBN;
+  const int pair = static_cast<int>(gridDim.y) - 1 - static_cast<int>(blockIdx.y);  // heavy first
+  const int n_kv_all = (n + L::kBN - 1) / L::kBN;
+  const int qt0 = 2 * pair, qt1 = 2 * pair + 1;
+  const int n0 = kCausal ? min(qt0 + 1, n_kv_all) : n_kv_all;  // key tiles seen by Q tile 0
+  const int n1 = kCausal ? min(qt1 + 1, n_kv_all) : n_kv_all;  // ... by Q tile 1 (n1 >= n0)
   const unsigned int err_fwd = kErrFwd;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(L::kQFull), 1);
-    for (int s = 0; s < S; ++s) {
-      mbar_init(bar(L::kKFull + s), 1);
-      mbar_init(bar(L::kKEmpty + s), 1);
-      mbar_init(bar(L::kVFull + s), 1);
-      mbar_init(bar(L::kVEmpty + s), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(L::kSFull + b), 1);
-      mbar_init(bar(L::kSFree + b), 4);  // one arrive per softmax warp
-    }
-    mbar_init(bar(L::kPFull), 4);
-    mbar_init(bar(L::kODone), 1);
-    mbar_init(bar(L::kDrain), 1);
+    for (int b = 0; b < L::kNumBars; ++b)
+      mbar_init(bar(b), (b == L::kPFull || b == L::kPFull + 1) ? 4u : 1u);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -118,216 +129,255 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_o);
-      bool ok = true;
-      int issued = 0;
-      mbar_arrive_expect_tx(bar(L::kQFull), L::kTile);
-      for (int db = 0; db < kDBlk; ++db)
-        tma_load_3d(sb + L::kOffQ + db * 16384, &tm_q, bar(L::kQFull), db * 64, qt * L::kBM, bh);
-      for (int t = 0; t < n_kv; ++t) {
-        const int s = t % S;
-        const uint32_t ph = (t / S) & 1;
-        if (!wait_bounded(bar(L::kKEmpty + s), ph ^ 1, limit_ns, abort_flag,
-                          err_fwd | kErrRoleLoad)) {
-          ok = false;
-          break;
+  // Registers: the block launches with 168 per thread (384 x 168 = 64512).
+  // Load / MMA / idle warps drop to 80, the two softmax warp groups rise to
+  // 200: 128 x 80 + 256 x 200 = 61440 <= 64512.
+  if (warp < 4) {
+    setmaxnreg_dec<L::kRegsOther>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_o);
+        const uint32_t err = err_fwd | kErrRoleLoad;
+        int nk = 0, nv = 0;
+        mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTile);
+        for (int db = 0; db < kDBlk; ++db) {
+          tma_load_3d(sb + L::kOffQ0 + db * 16384, &tm_q, bar(L::kQFull), db * 64, qt0 * L::kBM, bh);
+          tma_load_3d(sb + L::kOffQ1 + db * 16384, &tm_q, bar(L::kQFull), db * 64, qt1 * L::kBM, bh);
         }
-        mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTile);
-        for (int db = 0; db < kDBlk; ++db)
-          tma_load_3d(sb + L::kOffK + s * L::kTile + db * 16384, &tm_k, bar(L::kKFull + s),
-                      db * 64, t * L::kBN, bh);
-        if (!wait_bounded(bar(L::kVEmpty + s), ph ^ 1, limit_ns, abort_flag,
-                          err_fwd | kErrRoleLoad)) {
-          ok = false;
-          issued = 2 * t + 1;
-          break;
+        for (int j = 0; j < n1; ++j) {
+          const int s = j % S;
+          const uint32_t ph = (j / S) & 1;
+          if (!wait_bounded(bar(L::kKEmpty + s), ph ^ 1, limit_ns, abort_flag, err)) break;
+          mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTile);
+          for (int db = 0; db < kDBlk; ++db)
+            tma_load_3d(sb + L::kOffK + s * L::kTile + db * 16384, &tm_k, bar(L::kKFull + s),
+                        db * 64, j * L::kBN, bh);
+          ++nk;
+          if (!wait_bounded(bar(L::kVEmpty + s), ph ^ 1, limit_ns, abort_flag, err)) break;
+          mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTile);
+          for (int db = 0; db < kDBlk; ++db)
+            tma_load_3d(sb + L::kOffV + s * L::kTile + db * 16384, &tm_v, bar(L::kVFull + s),
+                        db * 64, j * L::kBN, bh);
+          ++nv;
         }
-        mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTile);
-        for (int db = 0; db < kDBlk; ++db)
-          tma_load_3d(sb + L::kOffV + s * L::kTile + db * 16384, &tm_v, bar(L::kVFull + s),
-                      db * 64, t * L::kBN, bh);
-        issued = 2 * t + 2;
+        if (*abort_flag) {
+          // let every copy already issued land before shared memory is released
+          drain_wait(bar(L::kQFull), 0, limit_ns);
+          for (int j = (nk > S ? nk - S : 0); j < nk; ++j)
+            drain_wait(bar(L::kKFull + j % S), (j / S) & 1, limit_ns);
+          for (int j = (nv > S ? nv - S : 0); j < nv; ++j)
+            drain_wait(bar(L::kVFull + j % S), (j / S) & 1, limit_ns);
+        }
       }
-      if (!ok) {
-        // let every copy already issued land before shared memory is released
-        drain_wait(bar(L::kQFull), 0, limit_ns);
-        const int nk = (issued + 1) / 2, nv = issued / 2;
-        for (int t = (nk > S ? nk - S : 0); t < nk; ++t)
-          drain_wait(bar(L::kKFull + t % S), (t / S) & 1, limit_ns);
-        for (int t = (nv > S ? nv - S : 0); t < nv; ++t)
-          drain_wait(bar(L::kVFull + t % S), (t / S) & 1, limit_ns);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t id_o = idesc_bf16_f32(128, D, false, true);
+        const uint32_t err = err_fwd | kErrRoleMma;
+        auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
+          const uint32_t qa = sb + (t ? L::kOffQ1 : L::kOffQ0);
+          const uint32_t ka = sb + L::kOffK + (j % S) * L::kTile;
+          const uint32_t d_tmem = tmem + (t ? L::kColS1 : L::kColS0);
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16_ss(d_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), id_s,
+                        kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(L::kSFull + t));
+        };
+        auto issue_pv = [&](int t, int j) {  // O_t += P_t V_j, P_t from TMEM
+          const uint32_t va = sb + L::kOffV + (j % S) * L::kTile;
+          const uint32_t d_tmem = tmem + (t ? L::kColO1 : L::kColO0);
+          const uint32_t a_tmem = tmem + (t ? L::kColS1 : L::kColS0);
+  #pragma unroll
+          for (int kk = 0; kk < L::kBN / 16; ++kk)
+            mma_bf16_ts(d_tmem, a_tmem + kk * 8, sw128_desc(va + kk * 2048, 16384, 1024), id_o,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+        };
+        bool ok = wait_bounded(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
+                  wait_bounded(bar(L::kKFull), 0, limit_ns, abort_flag, err);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          tc_commit(bar(L::kKEmpty));
+        }
+        for (int j = 0; ok && j < n1; ++j) {
+          const int s = j % S;
+          if (!wait_bounded(bar(L::kVFull + s), (j / S) & 1, limit_ns, abort_flag, err)) break;
+          if (j < n0) {
+            if (!wait_bounded(bar(L::kPFull + 0), j & 1, limit_ns, abort_flag, err)) break;
+            tc_fence_after();
+            issue_pv(0, j);
+            if (j == n0 - 1) tc_commit(bar(L::kOFinal + 0));
+          }
+          const bool next = j + 1 < n1;
+          const int s1 = (j + 1) % S;
+          if (next) {
+            if (!wait_bounded(bar(L::kKFull + s1), ((j + 1) / S) & 1, limit_ns, abort_flag, err))
+              break;
+            tc_fence_after();
+            if (j + 1 < n0) issue_s(0, j + 1);
+          }
+          if (!wait_bounded(bar(L::kPFull + 1), j & 1, limit_ns, abort_flag, err)) break;
+          tc_fence_after();
+          issue_pv(1, j);
+          if (j == n1 - 1) tc_commit(bar(L::kOFinal + 1));
+          tc_commit(bar(L::kVEmpty + s));
+          if (next) {
+            issue_s(1, j + 1);
+            tc_commit(bar(L::kKEmpty + s1));
+          }
+        }
+        // every MMA issued above must finish before TMEM / smem are released
+        tc_commit(bar(L::kDrain));
+        drain_wait(bar(L::kDrain), 0, limit_ns);
       }
+      __syncwarp();
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t id_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t err = err_fwd | kErrRoleMma;
-      auto issue_s = [&](int t) -> bool {
-        const int s = t % S;
-        const int b = t & 1;
-        if (!wait_bounded(bar(L::kKFull + s), (t / S) & 1, limit_ns, abort_flag, err)) return false;
-        if (!wait_bounded(bar(L::kSFree + b), ((t >> 1) & 1) ^ 1, limit_ns, abort_flag, err))
-          return false;
-        tc_fence_after();
-        const uint32_t qa = sb + L::kOffQ;
-        const uint32_t ka = sb + L::kOffK + s * L::kTile;
-        const uint32_t d_tmem = tmem + (b ? L::kColS1 : L::kColS0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(d_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), id_s,
-                      kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar(L::kSFull + b));
-        tc_commit(bar(L::kKEmpty + s));
-        return true;
-      };
-      bool ok = wait_bounded(bar(L::kQFull), 0, limit_ns, abort_flag, err) && issue_s(0);
-      for (int t = 0; ok && t < n_kv; ++t) {
-        if (t + 1 < n_kv && !issue_s(t + 1)) break;
-        const int s = t % S;
-        if (!wait_bounded(bar(L::kPFull), t & 1, limit_ns, abort_flag, err)) break;
-        if (!wait_bounded(bar(L::kVFull + s), (t / S) & 1, limit_ns, abort_flag, err)) break;
-        tc_fence_after();
-        const uint32_t pa = sb + L::kOffP;
-        const uint32_t va = sb + L::kOffV + s * L::kTile;
-#pragma unroll
-        for (int kk = 0; kk < L::kBN / 16; ++kk) {
-          const uint32_t poff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + L::kColO, sw128_desc(pa + poff, 16, 1024),
-                      sw128_desc(va + kk * 2048, 16384, 1024), id_o, (t > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar(L::kODone));
-        tc_commit(bar(L::kVEmpty + s));
-      }
-      // every MMA issued above must finish before TMEM / smem are released
-      tc_commit(bar(L::kDrain));
-      drain_wait(bar(L::kDrain), 0, limit_ns);
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc<L::kRegsSoftmax>();
     // ------------------------------------------------- softmax / epilogue
-    const int r = threadIdx.x - 128;  // row inside the tile == TMEM lane
+    const int t = (warp >= 8) ? 1 : 0;         // which Q tile
+    const int r = threadIdx.x - 128 - 128 * t;  // row inside the tile == TMEM lane
+    const int qt = qt0 + t;
+    const int n_t = t ? n1 : n0;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + (t ? L::kColS1 : L::kColS0);
+    const uint32_t o_addr = tmem + lane_off + (t ? L::kColO1 : L::kColO0);
     const uint32_t err = err_fwd | kErrRoleSoftmax;
-    float m_run = -INFINITY;  // running max of scale*log2(e)*s
+    const bool neg_scale = scale_log2 < 0.f;
+    const uint32_t masked_bits = __float_as_uint(neg_scale ? INFINITY : -INFINITY);
+    float m_run = -INFINITY;  // running (possibly stale) max of scale*log2(e)*s
     float l_run = 0.f;        // running sum of 2^(x - m_run)
     bool ok = true;
-    for (int t = 0; t < n_kv; ++t) {
-      const int b = t & 1;
-      if (!wait_bounded(bar(L::kSFull + b), (t >> 1) & 1, limit_ns, abort_flag, err)) {
+    for (int j = 0; j < n_t; ++j) {
+      if (!wait_bounded_warp(bar(L::kSFull + t), j & 1, limit_ns, abort_flag, err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float x[128];
-      {
-        const uint32_t sa = tmem + lane_off + (b ? L::kColS1 : L::kColS0);
-        uint32_t u[128];
+      uint32_t u[128];  // raw fp32 scores of this row
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld_32x32b_x32(sa + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 128; ++i) x[i] = __uint_as_float(u[i]) * scale_log2;
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::kSFree + b));
-
-      // mask: causal diagonal tile (key > query) and keys past the end
+      for (int c = 0; c < 4; ++c)
+        tmem_ld_32x32b_x32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
+      tmem_wait_ld();
+      // mask: causal diagonal tile (key > query) and keys past the end.  A
+      // masked score becomes the value that scales to -inf.
       int lim = L::kBN;
-      if (kCausal && t == qt) lim = r + 1;
-      const int rem = n - t * L::kBN;
+      if (kCausal && j == qt) lim = r + 1;
+      const int rem = n - j * L::kBN;
       if (rem < lim) lim = rem;
       if (lim < L::kBN) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = (c < lim) ? x[c] : -INFINITY;
+        for (int c = 0; c < 128; ++c) u[c] = (c < lim) ? u[c] : masked_bits;
       }
-      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+      // row max of scale*log2(e)*s: the max of s, or its min for a negative scale
+      float mx0 = __uint_as_float(u[0]), mx1 = __uint_as_float(u[1]);
+      float mx2 = __uint_as_float(u[2]), mx3 = __uint_as_float(u[3]);
+      if (neg_scale) {
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, x[c]);
-        mx1 = fmaxf(mx1, x[c + 1]);
-        mx2 = fmaxf(mx2, x[c + 2]);
-        mx3 = fmaxf(mx3, x[c + 3]);
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fminf(mx0, __uint_as_float(u[c]));
+          mx1 = fminf(mx1, __uint_as_float(u[c + 1]));
+          mx2 = fminf(mx2, __uint_as_float(u[c + 2]));
+          mx3 = fminf(mx3, __uint_as_float(u[c + 3]));
+        }
+        mx0 = fminf(fminf(mx0, mx1), fminf(mx2, mx3));
+      } else {
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fmaxf(mx0, __uint_as_float(u[c]));
+          mx1 = fmaxf(mx1, __uint_as_float(u[c + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(u[c + 2]));
+          mx3 = fmaxf(mx3, __uint_as_float(u[c + 3]));
+        }
+        mx0 = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
       }
-      const float m_new = fmaxf(m_run, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
-      const float alpha = ex2_approx(m_run - m_new);
-      uint32_t pk[64];
+      const float m_tile = mx0 * scale_log2;
+      const bool move = m_tile > m_run + L::kRescaleThreshold;
+      const float alpha = move ? ex2_approx(m_run - m_tile) : 1.0f;
+      if (move) m_run = m_tile;
+      const float neg_m = -m_run;
       float sum0 = 0.f, sum1 = 0.f;
+      // warp-uniform branch: both paths end in tcgen05.st, which every lane of
+      // the warp must execute together (a lane with lim == 128 masks nothing)
+      if (__any_sync(0xffffffffu, lim < L::kBN)) {
+        // masked tile: a masked key's probability is exactly 0 (also for a
+        // zero scale, where the -inf * 0 product would not be -inf)
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2_approx(x[c] - m_new);
-        const float p1 = ex2_approx(x[c + 1] - m_new);
-        sum0 += p0;
-        sum1 += p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int c = q * 32 + e;
+            float p0 = ex2_approx(fmaf(__uint_as_float(u[c]), scale_log2, neg_m));
+            float p1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), scale_log2, neg_m));
+            p0 = (c < lim) ? p0 : 0.f;
+            p1 = (c + 1 < lim) ? p1 : 0.f;
+            sum0 += p0;
+            sum1 += p1;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_32x32b_x16(s_addr + q * 16, pk);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {  // 32 keys -> 16 packed bf16 pairs -> TMEM
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(u[q * 32 + e]), scale_log2, neg_m));
+            const float p1 =
+                ex2_approx(fmaf(__uint_as_float(u[q * 32 + e + 1]), scale_log2, neg_m));
+            sum0 += p0;
+            sum1 += p1;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_32x32b_x16(s_addr + q * 16, pk);
+        }
       }
       l_run = l_run * alpha + (sum0 + sum1);
-      m_run = m_new;
-
-      if (t > 0) {
-        // PV of the previous tile must be done: it reads P and accumulates O
-        if (!wait_bounded(bar(L::kODone), (t - 1) & 1, limit_ns, abort_flag, err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-          const uint32_t oa = tmem + lane_off + L::kColO;
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t u[32];
-            tmem_ld_32x32b_x32(oa + c * 32, u);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld_32x32b_x32(o_addr + c * 32, u);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-            tmem_st_32x32b_x32(oa + c * 32, u);
-          }
-          tmem_wait_st();
+          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st_32x32b_x32(o_addr + c * 32, u);
         }
       }
-      // P tile: K-major, 128-byte swizzle, two 64-key blocks of 16 KiB
-      {
-        const uint32_t prow = sb + L::kOffP + r * 128;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t addr = prow + (j >> 3) * 16384 + ((((j & 7) ^ (r & 7))) << 4);
-          st_shared_v4(addr, pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        }
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::kPFull));
+      if (lane == 0) mbar_arrive(bar(L::kPFull + t));
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = wait_bounded(bar(L::kODone), (n_kv - 1) & 1, limit_ns, abort_flag,
+    if (ok) ok = wait_bounded_warp(bar(L::kOFinal + t), 0, limit_ns, abort_flag,
                               err_fwd | kErrRoleEpilogue);
+    const uint32_t stage = sb + (t ? L::kOffQ1 : L::kOffQ0);  // Q_t is dead: stage O_t there
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
-      const uint32_t oa = tmem + lane_off + L::kColO;
-      const uint32_t orow = sb + L::kOffQ + r * 128;  // Q tile is dead: stage O there
+      const uint32_t orow = stage + r * 128;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
-        tmem_ld_32x32b_x32(oa + c * 32, u);
+        tmem_ld_32x32b_x32(o_addr + c * 32, u);
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int j = c * 4 + q;  // 16-byte chunk index within the row
-          const uint32_t addr = orow + (j >> 3) * 16384 + ((((j & 7) ^ (r & 7))) << 4);
+          const int jj = c * 4 + q;  // 16-byte chunk index within the row
+          const uint32_t addr = orow + (jj >> 3) * 16384 + ((((jj & 7) ^ (r & 7))) << 4);
           st_shared_v4(addr,
                        pack_bf16x2(__uint_as_float(u[8 * q + 0]) * inv_l,
                                    __uint_as_float(u[8 * q + 1]) * inv_l),
@@ -340,14 +390,16 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
       const int row = qt * L::kBM + r;
-      if (row < n) lse_out[static_cast<size_t>(bh) * n + row] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+      if (row < n)
+        lse_out[static_cast<size_t>(bh) * n + row] =
+            (m_run + __log2f(l_run)) * 0.69314718055994530942f;
       fence_proxy_async_smem();
     }
     tc_fence_before();
-    named_barrier_sync(1, 128);  // every softmax warp reaches this, ok or not
-    if (threadIdx.x == 128 && ok && !*abort_flag) {
+    named_barrier_sync(1 + t, 128);  // every warp of this tile reaches this, ok or not
+    if (r == 0 && ok && !*abort_flag && qt * L::kBM < n) {
       for (int db = 0; db < kDBlk; ++db)
-        tma_store_3d(&tm_o, sb + L::kOffQ + db * 16384, db * 64, qt * L::kBM, bh);
+        tma_store_3d(&tm_o, stage + db * 16384, db * 64, qt * L::kBM, bh);
       bulk_commit_group();
       bulk_wait_group_0();
     }

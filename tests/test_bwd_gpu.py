@@ -118,3 +118,12 @@ def test_bwd_poisoned_outputs_fully_written():
     fa.check_device_error()
     for t in (dq, dk, dv):
         assert torch.isfinite(t.float()).all()
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.09])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_any_finite_scale(scale, causal):
+    w = Workload("scale", 1, 2, 300, 64, seed_base=14)
+    x = make_inputs(w, DEV)
+    _, _, grads = _fwd_bwd(x, causal, scale)
+    _check(x, grads, causal, scale, [(0, 0), (0, 1)])

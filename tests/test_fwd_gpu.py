@@ -137,3 +137,12 @@ def test_fwd_writes_nothing_past_the_end():
     fa.check_device_error()
     assert torch.all(big[:, :, 200:] == 7.0)
     assert torch.all(lse_big[200:] == 5.0)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.09, 0.5])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_any_finite_scale(scale, causal):
+    """Zero and negative scales are finite values the API accepts."""
+    w = Workload("scale", 1, 2, 300, 128, seed_base=13)
+    x = make_inputs(w, DEV, with_do=False)
+    _run_and_check(x["q"], x["k"], x["v"], causal, scale)
