@@ -77,27 +77,29 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------- dQ convert
+// The accumulator holds each 128-row tile as [D/4 column groups][128 rows][4];
+// thread (p, row) reads column groups 2p and 2p+1 of its row (consecutive
+// threads take consecutive rows: coalesced reads) and writes 8 bf16 of dQ.
 template <int D>
 __global__ void __launch_bounds__(256)
     dq_convert_kernel(const float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dq, int bh_count,
                       int n, int np, float scale) {
-  const long long i8 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;  // 8 elements
-  const long long total8 = static_cast<long long>(bh_count) * n * D / 8;
-  if (i8 >= total8) return;
-  const long long e = i8 * 8;
-  const long long row = e / D;  // bh * n + r
-  const int c = static_cast<int>(e % D);
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long rows = static_cast<long long>(bh_count) * n;
+  if (idx >= rows * (D / 8)) return;
+  const int p = static_cast<int>(idx / rows);  // group of 8 columns
+  const long long row = idx % rows;            // bh * n + r
   const long long bh = row / n;
-  const long long r = row % n;
-  const float* src = dq_acc + (bh * np + r) * D + c;
-  const float4 a = *reinterpret_cast<const float4*>(src);
-  const float4 b = *reinterpret_cast<const float4*>(src + 4);
+  const int r = static_cast<int>(row % n);
+  const float* tile = dq_acc + (bh * (np / 128) + r / 128) * 128LL * D;
+  const float4 a = *reinterpret_cast<const float4*>(tile + (2 * p) * 512 + (r % 128) * 4);
+  const float4 b = *reinterpret_cast<const float4*>(tile + (2 * p + 1) * 512 + (r % 128) * 4);
   uint4 w;
   w.x = pack_bf16x2(a.x * scale, a.y * scale);
   w.y = pack_bf16x2(a.z * scale, a.w * scale);
   w.z = pack_bf16x2(b.x * scale, b.y * scale);
   w.w = pack_bf16x2(b.z * scale, b.w * scale);
-  *reinterpret_cast<uint4*>(dq + e) = w;
+  *reinterpret_cast<uint4*>(dq + row * D + 8 * p) = w;
 }
 
 }  // namespace fa

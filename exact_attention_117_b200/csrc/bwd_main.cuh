@@ -22,7 +22,9 @@
 // dK_j and dV_j accumulate in TMEM and are written once by this CTA (no
 // atomics), staged through shared memory and stored with TMA; dQ_i partial
 // products are read out of TMEM by a separate warp group and added into the
-// fp32 accumulator with vector atomic adds.
+// fp32 accumulator with vector atomic adds.  The accumulator keeps each
+// 128-row tile as [D/4 column groups][128 rows][4 floats] so that those adds
+// are coalesced.
 //
 // Warp roles (384 threads): warp 0 TMA producer; warp 1 TMEM allocator and MMA
 // issuer; warps 4-7 compute P^T / dS^T (thread = key row) and write dK, dV;
@@ -400,10 +402,14 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::kDqFree));
-      float* dst = dq_acc + (static_cast<size_t>(bh) * np + static_cast<size_t>(i) * 128 + c) * D;
+      // accumulator tile layout [column group of 4][128 rows][4]: lane c's four
+      // columns sit next to lane c+1's, so one warp-wide vector add covers 512
+      // contiguous bytes (full sectors)
+      float* dst = dq_acc + (static_cast<size_t>(bh) * n_q + static_cast<size_t>(i)) * 128 * D +
+                   static_cast<size_t>(c) * 4;
 #pragma unroll
       for (int q = 0; q < D / 4; ++q)
-        red_add_v4(dst + 4 * q, __uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+        red_add_v4(dst + q * 512, __uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
                    __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
     }
   }

@@ -283,22 +283,22 @@ __global__ void __launch_bounds__(384, 1)
       float mx2 = __uint_as_float(u[2]), mx3 = __uint_as_float(u[3]);
       if (neg_scale) {
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fminf(mx0, __uint_as_float(u[c]));
-          mx1 = fminf(mx1, __uint_as_float(u[c + 1]));
-          mx2 = fminf(mx2, __uint_as_float(u[c + 2]));
-          mx3 = fminf(mx3, __uint_as_float(u[c + 3]));
+        for (int c = 4; c < 128; c += 8) {
+          mx0 = fmin3(mx0, __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
+          mx1 = fmin3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
+          mx2 = fmin3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
+          mx3 = fmin3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
         }
-        mx0 = fminf(fminf(mx0, mx1), fminf(mx2, mx3));
+        mx0 = fminf(fmin3(mx0, mx1, mx2), mx3);
       } else {
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, __uint_as_float(u[c]));
-          mx1 = fmaxf(mx1, __uint_as_float(u[c + 1]));
-          mx2 = fmaxf(mx2, __uint_as_float(u[c + 2]));
-          mx3 = fmaxf(mx3, __uint_as_float(u[c + 3]));
+        for (int c = 4; c < 128; c += 8) {
+          mx0 = fmax3(mx0, __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
+          mx1 = fmax3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
+          mx2 = fmax3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
+          mx3 = fmax3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
         }
-        mx0 = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        mx0 = fmaxf(fmax3(mx0, mx1, mx2), mx3);
       }
       const float m_tile = mx0 * scale_log2;
       const bool move = m_tile > m_run + L::kRescaleThreshold;
@@ -328,14 +328,17 @@ __global__ void __launch_bounds__(384, 1)
           tmem_st_32x32b_x16(s_addr + q * 16, pk);
         }
       } else {
+        // one exponential in four runs on the FMA pipe (exp2_poly3), the rest on
+        // the MUFU unit, so that neither pipe paces the tile alone
 #pragma unroll
         for (int q = 0; q < 4; ++q) {  // 32 keys -> 16 packed bf16 pairs -> TMEM
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(u[q * 32 + e]), scale_log2, neg_m));
-            const float p1 =
-                ex2_approx(fmaf(__uint_as_float(u[q * 32 + e + 1]), scale_log2, neg_m));
+            const float a0 = fmaf(__uint_as_float(u[q * 32 + e]), scale_log2, neg_m);
+            const float a1 = fmaf(__uint_as_float(u[q * 32 + e + 1]), scale_log2, neg_m);
+            const float p0 = ex2_approx(a0);
+            const float p1 = ((e & 3) == 2) ? exp2_poly3(a1) : ex2_approx(a1);
             sum0 += p0;
             sum1 += p1;
             pk[e >> 1] = pack_bf16x2(p0, p1);

@@ -82,9 +82,10 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
                  int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
- * Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator
- * [B, H, Np, d] plus two fp32 per-row vectors [B, H, Np] (D = rowsum(dO * O)
- * and the log2-domain LSE), with Np = N rounded up to a multiple of 128.
+ * Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator of
+ * B*H*Np*d floats (internal tile layout) plus two fp32 per-row vectors
+ * [B, H, Np] (D = rowsum(dO * O) and the log2-domain LSE), with Np = N
+ * rounded up to a multiple of 128.
  * Returns 0 if the arguments are invalid.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int H, int N, int d);
