@@ -332,6 +332,13 @@ fa_status fa_check_device_error(void* stream, unsigned int* detail) {
   return word ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
 }
 
+fa_status fa_selftest_watchdog(unsigned int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return FA_ERR_SHAPE;
+  fa::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_ms) * 1000000ull);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 const char* fa_status_string(fa_status s) {
   switch (s) {
     case FA_OK: return "ok";

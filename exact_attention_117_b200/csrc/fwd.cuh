@@ -328,8 +328,6 @@ __global__ void __launch_bounds__(384, 1)
           tmem_st_32x32b_x16(s_addr + q * 16, pk);
         }
       } else {
-        // one exponential in four runs on the FMA pipe (exp2_poly3), the rest on
-        // the MUFU unit, so that neither pipe paces the tile alone
 #pragma unroll
         for (int q = 0; q < 4; ++q) {  // 32 keys -> 16 packed bf16 pairs -> TMEM
           uint32_t pk[16];
@@ -338,7 +336,7 @@ __global__ void __launch_bounds__(384, 1)
             const float a0 = fmaf(__uint_as_float(u[q * 32 + e]), scale_log2, neg_m);
             const float a1 = fmaf(__uint_as_float(u[q * 32 + e + 1]), scale_log2, neg_m);
             const float p0 = ex2_approx(a0);
-            const float p1 = ((e & 3) == 2) ? exp2_poly3(a1) : ex2_approx(a1);
+            const float p1 = ex2_approx(a1);
             sum0 += p0;
             sum1 += p1;
             pk[e >> 1] = pack_bf16x2(p0, p1);

@@ -278,24 +278,6 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return r;
 }
 
-// 2^x on the FMA pipe, for x <= 64 (anything below -126 returns a value
-// <= 2^-126, i.e. an fp32 denormal or zero).  Cody-Waite style split
-// x = n + f with n = round(x) (the 1.5 * 2^23 addition rounds to nearest and
-// leaves n in the low mantissa bits) and f in [-0.5, 0.5]; 2^f by a cubic
-// that minimises the maximum relative error on [-0.5, 0.5] (coefficients from
-// a Remez exchange, gen_exp2_poly.py; max relative error 7.5e-5, well below
-// the bf16 rounding the probabilities get); 2^n is added into the exponent
-// field.
-__device__ __forceinline__ float exp2_poly3(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.0551716685f, f, 0.242611125f);
-  p = fmaf(p, f, 0.693260968f);
-  p = fmaf(p, f, 0.999928057f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

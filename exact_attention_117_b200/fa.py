@@ -56,6 +56,8 @@ def load() -> ctypes.CDLL:
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
     lib.fa_check_device_error.restype = i
     lib.fa_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    lib.fa_selftest_watchdog.restype = i
+    lib.fa_selftest_watchdog.argtypes = [ctypes.c_uint, vp]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_status_string.argtypes = [i]
     lib.fa_timing_begin.restype = i
@@ -186,6 +188,11 @@ def check_device_error(stream=None):
     st = load().fa_check_device_error(_stream_ptr(stream), ctypes.byref(detail))
     if st != FA_OK:
         raise FaError(st, f"device error word 0x{detail.value:x}")
+
+
+def selftest_watchdog(limit_ms: int = 200, stream=None):
+    """Launch the bounded-wait self-test kernel (see fa_selftest_watchdog)."""
+    _check(load().fa_selftest_watchdog(int(limit_ms), _stream_ptr(stream)), "fa_selftest_watchdog")
 
 
 class KernelTimer:

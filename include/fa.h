@@ -150,6 +150,18 @@ FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, con
  */
 FA_API fa_status fa_check_device_error(void* stream, unsigned int* detail);
 
+/*
+ * Self-test of the device-side wait limit (the pages have no counterpart: it
+ * checks this library's failure detection).  Launches one 32-thread kernel on
+ * `stream` that waits on a barrier no thread ever arrives on, with a limit of
+ * `limit_ms` milliseconds (1..2000).  The wait gives up, records the fact in
+ * the device error word and the kernel returns, so the next
+ * fa_check_device_error reports FA_ERR_DEVICE_TIMEOUT (detail bit 1 << 15)
+ * and the context stays usable.  Returns FA_ERR_SHAPE for a limit out of
+ * range, FA_ERR_CUDA if the launch fails.
+ */
+FA_API fa_status fa_selftest_watchdog(unsigned int limit_ms, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FA_API const char* fa_status_string(fa_status s);
 
