@@ -20,6 +20,7 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxSplits = 64;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s per bounded wait
 
 // ------------------------------------------------------------ TMA encoding
@@ -142,24 +143,27 @@ BwdWorkspace bwd_workspace_layout(void* base, int B, int H, int N, int d) {
   return w;
 }
 
-template <int D, bool C>
+template <int D, bool C, bool kSplit>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mo, float* lse, int BH, int N, float scale_log2,
-                     cudaStream_t st) {
+                     cudaStream_t st, int num_splits = 1, float* part_o = nullptr,
+                     float* part_lse = nullptr) {
   using L = fa::FwdLayout<D>;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return FA_ERR_CUDA;
   if (!attr_set[dev]) {
-    if (!set_smem(fa::fwd_kernel<D, C>, L::kSmemAlloc)) return FA_ERR_CUDA;
+    if (!set_smem(fa::fwd_kernel<D, C, kSplit>, L::kSmemAlloc)) return FA_ERR_CUDA;
     attr_set[dev] = true;
   }
   const int q_tiles = (N + L::kBM - 1) / L::kBM;
-  dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>((q_tiles + 1) / 2));  // 2 Q tiles per CTA
+  // 2 Q tiles per CTA; one CTA per split of the key range in split mode
+  dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>((q_tiles + 1) / 2),
+            static_cast<unsigned>(kSplit ? num_splits : 1));
   {
     LaunchTimer timer(st, FA_KERNEL_FWD);
-    fa::fwd_kernel<D, C><<<grid, 384, L::kSmemAlloc, st>>>(mq, mk, mv, mo, lse, N, scale_log2,
-                                                          kWaitLimitNs);
+    fa::fwd_kernel<D, C, kSplit><<<grid, 384, L::kSmemAlloc, st>>>(
+        mq, mk, mv, mo, lse, N, scale_log2, kWaitLimitNs, num_splits, part_o, part_lse);
   }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -226,10 +230,66 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
-    return causal ? launch_fwd<64, true>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
-                  : launch_fwd<64, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
-  return causal ? launch_fwd<128, true>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
-                : launch_fwd<128, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
+    return causal ? launch_fwd<64, true, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
+                  : launch_fwd<64, false, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
+  return causal ? launch_fwd<128, true, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
+                : launch_fwd<128, false, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits) {
+  if (check_common(B, H, N, d, 1.0f) != FA_OK) return 0;
+  if (num_splits < 1 || num_splits > kMaxSplits) return 0;
+  const size_t rows = static_cast<size_t>(num_splits) * B * H * round_up(static_cast<size_t>(N), 128);
+  return rows * static_cast<size_t>(d + 1) * sizeof(float);  // partial O, then partial LSE
+}
+
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int N, int d, int causal, float scale, int num_splits,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (num_splits < 1 || num_splits > kMaxSplits) return FA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGN;
+  const size_t need = fa_fwd_splitkv_workspace_size(B, H, N, d, num_splits);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGN;
+  const int bh = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
+      !encode_bf16_3d(&mv, v, d, N, bh, 128))
+    return FA_ERR_CUDA;
+  float* part_o = static_cast<float*>(workspace);
+  float* part_lse =
+      part_o + static_cast<size_t>(num_splits) * bh * round_up(static_cast<size_t>(N), 128) * d;
+  const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fa_status r;
+  if (d == 64)
+    r = causal ? launch_fwd<64, true, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s, num_splits,
+                                            part_o, part_lse)
+               : launch_fwd<64, false, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
+                                             num_splits, part_o, part_lse);
+  else
+    r = causal ? launch_fwd<128, true, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
+                                             num_splits, part_o, part_lse)
+               : launch_fwd<128, false, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
+                                              num_splits, part_o, part_lse);
+  if (r != FA_OK) return r;
+  {
+    LaunchTimer timer(s, FA_KERNEL_FWD_COMBINE);
+    const long long threads = static_cast<long long>(bh) * N * (d / 8);
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    if (d == 64)
+      fa::splitkv_combine_kernel<64><<<blocks, 256, 0, s>>>(
+          part_o, part_lse, static_cast<__nv_bfloat16*>(o), lse, bh, N, num_splits);
+    else
+      fa::splitkv_combine_kernel<128><<<blocks, 256, 0, s>>>(
+          part_o, part_lse, static_cast<__nv_bfloat16*>(o), lse, bh, N, num_splits);
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

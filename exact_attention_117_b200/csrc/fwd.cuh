@@ -43,6 +43,8 @@
 // converted back to natural log.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 
 namespace fa {
@@ -86,11 +88,18 @@ struct FwdLayout {
   static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= 384 * kLaunchRegs, "register split");
 };
 
-template <int D, bool kCausal>
+// kSplit: the CTA covers only the key tiles of split blockIdx.z (a contiguous
+// range of ceil(n_kv / num_splits) tiles) and writes, instead of O and LSE,
+// fp32 partial results: O_s = u_s / l_s in the tile layout [D/4 column
+// groups][128 rows][4] of part_o, and LSE_s = m_s + log2 l_s (base 2) in
+// part_lse; a split that sees no key of a row writes O_s = 0, LSE_s = -inf.
+// splitkv_combine_kernel merges the splits.
+template <int D, bool kCausal, bool kSplit>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-               float* __restrict__ lse_out, int n, float scale_log2, uint64_t limit_ns) {
+               float* __restrict__ lse_out, int n, float scale_log2, uint64_t limit_ns,
+               int num_splits, float* __restrict__ part_o, float* __restrict__ part_lse) {
   using L = FwdLayout<D>;
   constexpr int S = L::kStages;
   constexpr int kDBlk = D / 64;  // 128-byte swizzle blocks per tile row
@@ -107,10 +116,20 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x;
   const int pair = static_cast<int>(gridDim.y) - 1 - static_cast<int>(blockIdx.y);  // heavy first
-  const int n_kv_all = (n + L::kBN - 1) / L::kBN;
+  const int n_kv_all = (n + L::kBN - 1) / L::kBN;  // also the number of Q tiles (Nq = Nk)
   const int qt0 = 2 * pair, qt1 = 2 * pair + 1;
-  const int n0 = kCausal ? min(qt0 + 1, n_kv_all) : n_kv_all;  // key tiles seen by Q tile 0
-  const int n1 = kCausal ? min(qt1 + 1, n_kv_all) : n_kv_all;  // ... by Q tile 1 (n1 >= n0)
+  // key tiles [kb, ke) of this CTA: all of them, or this split's share
+  int kb = 0, ke = n_kv_all;
+  if (kSplit) {
+    const int chunk = (n_kv_all + num_splits - 1) / num_splits;
+    kb = static_cast<int>(blockIdx.z) * chunk;
+    ke = min(kb + chunk, n_kv_all);
+  }
+  const int end0 = kCausal ? min(qt0 + 1, n_kv_all) : n_kv_all;  // causal end, Q tile 0
+  const int end1 = kCausal ? min(qt1 + 1, n_kv_all) : n_kv_all;  // causal end, Q tile 1
+  // key tiles each Q tile processes here, from kb on (n1 >= n0; a split may have 0)
+  const int n0 = max(0, min(ke, end0) - kb);
+  const int n1 = max(0, min(ke, end1) - kb);
   const unsigned int err_fwd = kErrFwd;
 
   if (threadIdx.x == 0) {
@@ -143,14 +162,15 @@ __global__ void __launch_bounds__(384, 1)
         tma_prefetch_desc(&tm_o);
         const uint32_t err = err_fwd | kErrRoleLoad;
         int nk = 0, nv = 0;
-        mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTile);
-        for (int db = 0; db < kDBlk; ++db) {
+        if (n1 > 0) mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTile);
+        for (int db = 0; n1 > 0 && db < kDBlk; ++db) {
           tma_load_3d(sb + L::kOffQ0 + db * 16384, &tm_q, bar(L::kQFull), db * 64, qt0 * L::kBM, bh);
           tma_load_3d(sb + L::kOffQ1 + db * 16384, &tm_q, bar(L::kQFull), db * 64, qt1 * L::kBM, bh);
         }
-        for (int j = 0; j < n1; ++j) {
-          const int s = j % S;
-          const uint32_t ph = (j / S) & 1;
+        for (int jj = 0; jj < n1; ++jj) {
+          const int j = kb + jj;  // key tile
+          const int s = jj % S;
+          const uint32_t ph = (jj / S) & 1;
           if (!wait_bounded(bar(L::kKEmpty + s), ph ^ 1, limit_ns, abort_flag, err)) break;
           mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTile);
           for (int db = 0; db < kDBlk; ++db)
@@ -164,7 +184,7 @@ __global__ void __launch_bounds__(384, 1)
                         db * 64, j * L::kBN, bh);
           ++nv;
         }
-        if (*abort_flag) {
+        if (*abort_flag && n1 > 0) {
           // let every copy already issued land before shared memory is released
           drain_wait(bar(L::kQFull), 0, limit_ns);
           for (int j = (nk > S ? nk - S : 0); j < nk; ++j)
@@ -179,9 +199,9 @@ __global__ void __launch_bounds__(384, 1)
         constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t id_o = idesc_bf16_f32(128, D, false, true);
         const uint32_t err = err_fwd | kErrRoleMma;
-        auto issue_s = [&](int t, int j) {  // S_t = Q_t K_j^T
+        auto issue_s = [&](int t, int jj) {  // S_t = Q_t K_j^T, key tile j = kb + jj
           const uint32_t qa = sb + (t ? L::kOffQ1 : L::kOffQ0);
-          const uint32_t ka = sb + L::kOffK + (j % S) * L::kTile;
+          const uint32_t ka = sb + L::kOffK + (jj % S) * L::kTile;
           const uint32_t d_tmem = tmem + (t ? L::kColS1 : L::kColS0);
   #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -191,47 +211,47 @@ __global__ void __launch_bounds__(384, 1)
           }
           tc_commit(bar(L::kSFull + t));
         };
-        auto issue_pv = [&](int t, int j) {  // O_t += P_t V_j, P_t from TMEM
-          const uint32_t va = sb + L::kOffV + (j % S) * L::kTile;
+        auto issue_pv = [&](int t, int jj) {  // O_t += P_t V_j, P_t from TMEM
+          const uint32_t va = sb + L::kOffV + (jj % S) * L::kTile;
           const uint32_t d_tmem = tmem + (t ? L::kColO1 : L::kColO0);
           const uint32_t a_tmem = tmem + (t ? L::kColS1 : L::kColS0);
   #pragma unroll
           for (int kk = 0; kk < L::kBN / 16; ++kk)
             mma_bf16_ts(d_tmem, a_tmem + kk * 8, sw128_desc(va + kk * 2048, 16384, 1024), id_o,
-                        (j > 0 || kk > 0) ? 1u : 0u);
+                        (jj > 0 || kk > 0) ? 1u : 0u);
         };
-        bool ok = wait_bounded(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
+        bool ok = n1 > 0 && wait_bounded(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
                   wait_bounded(bar(L::kKFull), 0, limit_ns, abort_flag, err);
         if (ok) {
           tc_fence_after();
-          issue_s(0, 0);
+          if (n0 > 0) issue_s(0, 0);
           issue_s(1, 0);
           tc_commit(bar(L::kKEmpty));
         }
-        for (int j = 0; ok && j < n1; ++j) {
-          const int s = j % S;
-          if (!wait_bounded(bar(L::kVFull + s), (j / S) & 1, limit_ns, abort_flag, err)) break;
-          if (j < n0) {
-            if (!wait_bounded(bar(L::kPFull + 0), j & 1, limit_ns, abort_flag, err)) break;
+        for (int jj = 0; ok && jj < n1; ++jj) {
+          const int s = jj % S;
+          if (!wait_bounded(bar(L::kVFull + s), (jj / S) & 1, limit_ns, abort_flag, err)) break;
+          if (jj < n0) {
+            if (!wait_bounded(bar(L::kPFull + 0), jj & 1, limit_ns, abort_flag, err)) break;
             tc_fence_after();
-            issue_pv(0, j);
-            if (j == n0 - 1) tc_commit(bar(L::kOFinal + 0));
+            issue_pv(0, jj);
+            if (jj == n0 - 1) tc_commit(bar(L::kOFinal + 0));
           }
-          const bool next = j + 1 < n1;
-          const int s1 = (j + 1) % S;
+          const bool next = jj + 1 < n1;
+          const int s1 = (jj + 1) % S;
           if (next) {
-            if (!wait_bounded(bar(L::kKFull + s1), ((j + 1) / S) & 1, limit_ns, abort_flag, err))
+            if (!wait_bounded(bar(L::kKFull + s1), ((jj + 1) / S) & 1, limit_ns, abort_flag, err))
               break;
             tc_fence_after();
-            if (j + 1 < n0) issue_s(0, j + 1);
+            if (jj + 1 < n0) issue_s(0, jj + 1);
           }
-          if (!wait_bounded(bar(L::kPFull + 1), j & 1, limit_ns, abort_flag, err)) break;
+          if (!wait_bounded(bar(L::kPFull + 1), jj & 1, limit_ns, abort_flag, err)) break;
           tc_fence_after();
-          issue_pv(1, j);
-          if (j == n1 - 1) tc_commit(bar(L::kOFinal + 1));
+          issue_pv(1, jj);
+          if (jj == n1 - 1) tc_commit(bar(L::kOFinal + 1));
           tc_commit(bar(L::kVEmpty + s));
           if (next) {
-            issue_s(1, j + 1);
+            issue_s(1, jj + 1);
             tc_commit(bar(L::kKEmpty + s1));
           }
         }
@@ -257,8 +277,9 @@ __global__ void __launch_bounds__(384, 1)
     float m_run = -INFINITY;  // running (possibly stale) max of scale*log2(e)*s
     float l_run = 0.f;        // running sum of 2^(x - m_run)
     bool ok = true;
-    for (int j = 0; j < n_t; ++j) {
-      if (!wait_bounded_warp(bar(L::kSFull + t), j & 1, limit_ns, abort_flag, err)) {
+    for (int jj = 0; jj < n_t; ++jj) {
+      const int j = kb + jj;  // key tile
+      if (!wait_bounded_warp(bar(L::kSFull + t), jj & 1, limit_ns, abort_flag, err)) {
         ok = false;
         break;
       }
@@ -345,7 +366,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       l_run = l_run * alpha + (sum0 + sum1);
-      if (j > 0 && __any_sync(0xffffffffu, move)) {
+      if (jj > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t u[32];
@@ -363,46 +384,79 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = wait_bounded_warp(bar(L::kOFinal + t), 0, limit_ns, abort_flag,
-                              err_fwd | kErrRoleEpilogue);
-    const uint32_t stage = sb + (t ? L::kOffQ1 : L::kOffQ0);  // Q_t is dead: stage O_t there
-    if (ok) {
-      tc_fence_after();
-      const float inv_l = 1.0f / l_run;
-      const uint32_t orow = stage + r * 128;
+    if (kSplit) {
+      // partial result of this split (rows of a Q tile past the last tile of
+      // the sequence do not exist in the partial buffers)
+      if (n_t > 0 && ok)
+        ok = wait_bounded_warp(bar(L::kOFinal + t), 0, limit_ns, abort_flag,
+                               err_fwd | kErrRoleEpilogue);
+      if (ok && qt < n_kv_all) {
+        const size_t tile_idx = (static_cast<size_t>(blockIdx.z) * gridDim.x + bh) * n_kv_all + qt;
+        float* po = part_o + tile_idx * 128 * D + r * 4;
+        if (n_t > 0) {
+          tc_fence_after();
+          const float inv_l = 1.0f / l_run;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld_32x32b_x32(o_addr + c * 32, u);
-        tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tmem_ld_32x32b_x32(o_addr + c * 32, u);
+            tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int jj = c * 4 + q;  // 16-byte chunk index within the row
-          const uint32_t addr = orow + (jj >> 3) * 16384 + ((((jj & 7) ^ (r & 7))) << 4);
-          st_shared_v4(addr,
-                       pack_bf16x2(__uint_as_float(u[8 * q + 0]) * inv_l,
-                                   __uint_as_float(u[8 * q + 1]) * inv_l),
-                       pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv_l,
-                                   __uint_as_float(u[8 * q + 3]) * inv_l),
-                       pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv_l,
-                                   __uint_as_float(u[8 * q + 5]) * inv_l),
-                       pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv_l,
-                                   __uint_as_float(u[8 * q + 7]) * inv_l));
+            for (int g = 0; g < 8; ++g)
+              *reinterpret_cast<float4*>(po + (c * 8 + g) * 512) =
+                  make_float4(__uint_as_float(u[4 * g]) * inv_l, __uint_as_float(u[4 * g + 1]) * inv_l,
+                              __uint_as_float(u[4 * g + 2]) * inv_l,
+                              __uint_as_float(u[4 * g + 3]) * inv_l);
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < D / 4; ++g)
+            *reinterpret_cast<float4*>(po + g * 512) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        part_lse[tile_idx * 128 + r] = (n_t > 0) ? m_run + __log2f(l_run) : -INFINITY;
       }
-      const int row = qt * L::kBM + r;
-      if (row < n)
-        lse_out[static_cast<size_t>(bh) * n + row] =
-            (m_run + __log2f(l_run)) * 0.69314718055994530942f;
-      fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    named_barrier_sync(1 + t, 128);  // every warp of this tile reaches this, ok or not
-    if (r == 0 && ok && !*abort_flag && qt * L::kBM < n) {
-      for (int db = 0; db < kDBlk; ++db)
-        tma_store_3d(&tm_o, stage + db * 16384, db * 64, qt * L::kBM, bh);
-      bulk_commit_group();
-      bulk_wait_group_0();
+    } else {
+      if (ok) ok = wait_bounded_warp(bar(L::kOFinal + t), 0, limit_ns, abort_flag,
+                                err_fwd | kErrRoleEpilogue);
+      const uint32_t stage = sb + (t ? L::kOffQ1 : L::kOffQ0);  // Q_t is dead: stage O_t there
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.0f / l_run;
+        const uint32_t orow = stage + r * 128;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld_32x32b_x32(o_addr + c * 32, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int jj = c * 4 + q;  // 16-byte chunk index within the row
+            const uint32_t addr = orow + (jj >> 3) * 16384 + ((((jj & 7) ^ (r & 7))) << 4);
+            st_shared_v4(addr,
+                         pack_bf16x2(__uint_as_float(u[8 * q + 0]) * inv_l,
+                                     __uint_as_float(u[8 * q + 1]) * inv_l),
+                         pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv_l,
+                                     __uint_as_float(u[8 * q + 3]) * inv_l),
+                         pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv_l,
+                                     __uint_as_float(u[8 * q + 5]) * inv_l),
+                         pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv_l,
+                                     __uint_as_float(u[8 * q + 7]) * inv_l));
+          }
+        }
+        const int row = qt * L::kBM + r;
+        if (row < n)
+          lse_out[static_cast<size_t>(bh) * n + row] =
+              (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      named_barrier_sync(1 + t, 128);  // every warp of this tile reaches this, ok or not
+      if (r == 0 && ok && !*abort_flag && qt * L::kBM < n) {
+        for (int db = 0; db < kDBlk; ++db)
+          tma_store_3d(&tm_o, stage + db * 16384, db * 64, qt * L::kBM, bh);
+        bulk_commit_group();
+        bulk_wait_group_0();
+      }
     }
   }
 
@@ -412,6 +466,62 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
+}
+
+// Merge of the split partial results, page "FlashAttention 为什么能节省显存并提速,
+// 是否改变注意力结果?", section 难点在于分块后softmax如何归一: blocks are brought to a
+// common max before they are added.  With LSE_s = m_s + log2 l_s and
+// O_s = u_s / l_s (base 2):  M = max_s LSE_s,  w_s = 2^(LSE_s - M)
+// (= 2^(m_s - M) l_s),  l = sum_s w_s,  O = sum_s w_s O_s / l
+// (= sum_s 2^(m_s - M) u_s / l),  LSE = M + log2 l, stored as natural log.
+// Thread (p, row) owns 8 columns of one row; consecutive threads take
+// consecutive rows so the partial reads are coalesced.
+template <int D>
+__global__ void __launch_bounds__(256)
+    splitkv_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                           __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int bh_count,
+                           int n, int num_splits) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long rows = static_cast<long long>(bh_count) * n;
+  if (idx >= rows * (D / 8)) return;
+  const int p = static_cast<int>(idx / rows);
+  const long long row = idx % rows;
+  const long long bh = row / n;
+  const int r = static_cast<int>(row % n);
+  const int n_tiles = (n + 127) / 128;
+  const size_t tiles_per_split = static_cast<size_t>(bh_count) * n_tiles;
+  const size_t tile = static_cast<size_t>(bh) * n_tiles + r / 128;
+  float m = -INFINITY;
+  for (int s = 0; s < num_splits; ++s)
+    m = fmaxf(m, part_lse[(s * tiles_per_split + tile) * 128 + r % 128]);
+  float l = 0.f;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < num_splits; ++s) {
+    const size_t t = s * tiles_per_split + tile;
+    const float ls = part_lse[t * 128 + r % 128];
+    if (ls == -INFINITY) continue;  // this split saw no key of the row
+    const float w = ex2_approx(ls - m);
+    l += w;
+    const float* po = part_o + t * 128 * D + (r % 128) * 4;
+    const float4 a = *reinterpret_cast<const float4*>(po + (2 * p) * 512);
+    const float4 b = *reinterpret_cast<const float4*>(po + (2 * p + 1) * 512);
+    acc[0] = fmaf(w, a.x, acc[0]);
+    acc[1] = fmaf(w, a.y, acc[1]);
+    acc[2] = fmaf(w, a.z, acc[2]);
+    acc[3] = fmaf(w, a.w, acc[3]);
+    acc[4] = fmaf(w, b.x, acc[4]);
+    acc[5] = fmaf(w, b.y, acc[5]);
+    acc[6] = fmaf(w, b.z, acc[6]);
+    acc[7] = fmaf(w, b.w, acc[7]);
+  }
+  const float inv = 1.0f / l;
+  uint4 out;
+  out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(o + row * D + 8 * p) = out;
+  if (p == 0) lse[row] = (m + __log2f(l)) * 0.69314718055994530942f;
 }
 
 }  // namespace fa

@@ -24,7 +24,7 @@ STATUS_NAMES = {
     4: "FA_ERR_ALIGN", 5: "FA_ERR_SCALE", 6: "FA_ERR_WORKSPACE", 7: "FA_ERR_CUDA",
     8: "FA_ERR_DEVICE_TIMEOUT", 9: "FA_ERR_STATE",
 }
-KERNELS = ("fwd", "bwd_pre", "bwd_main", "bwd_dq")
+KERNELS = ("fwd", "bwd_pre", "bwd_main", "bwd_dq", "fwd_combine")
 
 _lib = None
 
@@ -48,6 +48,10 @@ def load() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_fwd.restype = i
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+    lib.fa_fwd_splitkv_workspace_size.restype = sz
+    lib.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_fwd_splitkv.restype = i
+    lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd.restype = i
@@ -129,6 +133,30 @@ def forward(q, k, v, causal: bool = False, scale: Optional[float] = None, out=No
     return out, lse
 
 
+def splitkv_workspace_size(B: int, H: int, N: int, d: int, num_splits: int) -> int:
+    return int(load().fa_fwd_splitkv_workspace_size(B, H, N, d, num_splits))
+
+
+def forward_splitkv(q, k, v, causal: bool = False, scale: Optional[float] = None,
+                    num_splits: int = 2, out=None, lse=None, workspace=None, stream=None):
+    """O, LSE through the split-KV forward (key range cut into ``num_splits``)."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = splitkv_workspace_size(B, H, N, d, num_splits)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(load().fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
+                                 int(bool(causal)), float(scale), int(num_splits),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream_ptr(stream)), "fa_fwd_splitkv")
+    return out, lse
+
+
 def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None,
              dq=None, dk=None, dv=None, workspace=None, stream=None):
     """dQ, dK, dV of sum(dO * O); the fp32 workspace is allocated here if not given."""
@@ -203,8 +231,8 @@ class KernelTimer:
         return self
 
     def __exit__(self, *exc):
-        ms = (ctypes.c_float * 4)()
-        cnt = (ctypes.c_int * 4)()
+        ms = (ctypes.c_float * len(KERNELS))()
+        cnt = (ctypes.c_int * len(KERNELS))()
         _check(load().fa_timing_end(ms, cnt), "fa_timing_end")
         self.ms = {k: float(ms[i]) for i, k in enumerate(KERNELS)}
         self.launches = {k: int(cnt[i]) for i, k in enumerate(KERNELS)}

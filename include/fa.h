@@ -82,6 +82,27 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
                  int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * Split-KV forward (page "FlashAttention 为什么能节省显存并提速,是否改变注意力结果?",
+ * section 难点在于分块后softmax如何归一: per-block statistics are brought to a
+ * common max and merged).  The key tiles are divided into num_splits
+ * contiguous ranges; one launch computes, for every Q tile and range, the
+ * normalised partial output and its logsumexp into the workspace, and a
+ * second launch merges the ranges: M = max_s LSE_s, w_s = exp(LSE_s - M),
+ * O = sum_s w_s O_s / sum_s w_s, LSE = M + ln sum_s w_s.  Same arguments,
+ * layouts and results as fa_fwd (up to rounding), plus:
+ *   num_splits : 1..64; ranges past the causal diagonal are skipped.  Useful
+ *                when B * H * ceil(N / 256) CTAs would not fill the GPU.
+ *   workspace  : device scratch of fa_fwd_splitkv_workspace_size bytes,
+ *                16-byte aligned, contents on entry irrelevant.
+ * Returns FA_ERR_SHAPE for num_splits out of range.
+ */
+FA_API size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits);
+FA_API fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int N, int d, int causal, float scale,
+                                int num_splits, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs: an fp32 dQ accumulator of
  * B*H*Np*d floats (internal tile layout) plus two fp32 per-row vectors
  * [B, H, Np] (D = rowsum(dO * O) and the log2-domain LSE), with Np = N
@@ -171,7 +192,8 @@ typedef enum {
   FA_KERNEL_BWD_PRE = 1,   /* backward: D = rowsum(dO*O), clears dQ  */
   FA_KERNEL_BWD_MAIN = 2,  /* backward: per-KV-tile main kernel      */
   FA_KERNEL_BWD_DQ = 3,    /* backward: dQ fp32 -> bf16              */
-  FA_KERNEL_COUNT = 4
+  FA_KERNEL_FWD_COMBINE = 4, /* split-KV forward: merge of the splits */
+  FA_KERNEL_COUNT = 5
 } fa_kernel_id;
 
 /*

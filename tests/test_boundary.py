@@ -114,10 +114,12 @@ def test_timing_state_machine(lib):
     assert lib.fa_timing_end(None, None) == 9
     assert lib.fa_timing_begin() == 0
     assert lib.fa_timing_begin() == 9
-    ms = (ctypes.c_float * 4)()
-    cnt = (ctypes.c_int * 4)()
+    from exact_attention_117_b200 import fa
+    nk = len(fa.KERNELS)  # FA_KERNEL_COUNT entries
+    ms = (ctypes.c_float * nk)()
+    cnt = (ctypes.c_int * nk)()
     assert lib.fa_timing_end(ms, cnt) == 0
-    assert list(cnt) == [0, 0, 0, 0]
+    assert list(cnt) == [0] * nk
 
 
 def test_binding_fails_loudly_without_library(monkeypatch):
@@ -126,3 +128,11 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(fa, "LIB_PATH", "/nonexistent/libfa_b200.so")
     with pytest.raises(RuntimeError, match="not built"):
         fa.load()
+
+
+def test_binding_kernel_list_matches_header():
+    from exact_attention_117_b200 import fa
+    with open(os.path.join(ROOT, "include", "fa.h")) as f:
+        text = f.read()
+    count = int(re.search(r"FA_KERNEL_COUNT\s*=\s*(\d+)", text).group(1))
+    assert count == len(fa.KERNELS)
