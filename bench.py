@@ -396,6 +396,89 @@ def run_ours(args, w, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def _time_device(fn, flush, stream, warmup=3, iters=10):
+    """Median CUDA-event time (ms) of fn(), L2 flushed before each timed call."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    times = []
+    for _ in range(iters):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    times.sort()
+    return times[len(times) // 2]
+
+
+def run_sweep(args):
+    """Supplementary measurements (one JSON line per case, not the headline line):
+    the B*H*N = 2^20 sweep (d in {64, 128}, N in 512..8192, causal and full,
+    forward and forward+backward) and the split-KV forward on few-head,
+    long-sequence problems where one CTA per Q-tile pair leaves SMs idle."""
+    import torch
+
+    from exact_attention_117_b200 import fa
+    from exact_attention_117_b200.workloads import Workload, make_inputs, sweep_workloads
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    peaks, _ = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+
+    def emit(case, tflops, ms):
+        print(json.dumps({"sweep": case, "tflops": round(tflops, 1), "ms": round(ms, 4),
+                          "pct_of_peak": round(100 * tflops / peak, 1)}), flush=True)
+
+    if args.sweep in ("all", "c5"):
+        for w in sweep_workloads():
+            x = make_inputs(w, dev)
+            o = torch.empty_like(x["q"])
+            lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+            g = [torch.empty_like(x["q"]) for _ in range(3)]
+            ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+            for causal in (True, False):
+                fwd_f, bwd_f = attention_flops(w.B, w.H, w.N, w.d, causal)
+
+                def fwd():
+                    fa.forward(x["q"], x["k"], x["v"], causal=causal, out=o, lse=lse, stream=stream)
+
+                def step():
+                    fwd()
+                    fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal,
+                                dq=g[0], dk=g[1], dv=g[2], workspace=ws, stream=stream)
+                tag = f"{w.name} {'causal' if causal else 'full'}"
+                ms = _time_device(fwd, flush, stream)
+                emit(f"{tag} fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
+                ms = _time_device(step, flush, stream)
+                emit(f"{tag} fwd+bwd", (fwd_f + bwd_f) / (ms * 1e-3) / 1e12, ms)
+            del x, o, lse, g, ws
+    if args.sweep in ("all", "splitkv"):
+        for B, H, N, causal in ((1, 1, 16384, False), (1, 1, 16384, True), (1, 2, 32768, False),
+                                (1, 4, 8192, False)):
+            w = Workload(f"few_heads_B{B}_H{H}_N{N}", B, H, N, 128, seed_base=500)
+            x = make_inputs(w, dev, with_do=False)
+            o = torch.empty_like(x["q"])
+            lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+            fwd_f, _ = attention_flops(B, H, N, 128, causal)
+            tag = f"{w.name} d=128 {'causal' if causal else 'full'}"
+            ms = _time_device(lambda: fa.forward(x["q"], x["k"], x["v"], causal=causal, out=o,
+                                                 lse=lse, stream=stream), flush, stream)
+            emit(f"{tag} fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
+            for splits in (2, 4, 8):
+                wsz = fa.splitkv_workspace_size(B, H, N, 128, splits)
+                wsp = torch.empty(wsz, dtype=torch.uint8, device=dev)
+                ms = _time_device(lambda: fa.forward_splitkv(
+                    x["q"], x["k"], x["v"], causal=causal, num_splits=splits, out=o, lse=lse,
+                    workspace=wsp, stream=stream), flush, stream)
+                emit(f"{tag} fwd split-KV x{splits}", fwd_f / (ms * 1e-3) / 1e12, ms)
+    fa.check_device_error(stream)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -406,7 +489,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--sweep", choices=["all", "c5", "splitkv"], default=None,
+                    help="supplementary per-case measurements instead of the headline line")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
 
     from exact_attention_117_b200.workloads import WORKLOADS
     w = WORKLOADS[args.workload]
