@@ -2,17 +2,24 @@
 //
 // K_j and V_j stay in shared memory for the whole CTA; the Q tiles i that see
 // key tile j (all of them, or i >= j under the causal mask, since Br = Bc)
-// stream through a two-stage ring together with dO_i, LSE_i and D_i.  Per Q
-// tile, with keys on the TMEM lanes (M = 128 keys):
+// stream through a two-stage ring, dO_i through its own ring.  Per Q tile,
+// with keys on the TMEM lanes (M = 128 keys):
 //
-//   S^T  = K_j Q_i^T            tcgen05, A = K_j (K-major), B = Q_i (K-major)
-//   dP^T = V_j dO_i^T           tcgen05, A = V_j (K-major), B = dO_i (K-major)
-//   P^T  = 2^(S^T*scale*log2e - LSE2_i)   one thread per key row, masked,
-//                               written back over S^T in TMEM as bf16
-//   dV_j += P^T dO_i            tcgen05, A = P^T (TMEM), B = dO_i (MN-major)
-//   dS^T = P^T o (dP^T - D_i)   written to shared memory as bf16
-//   dK_j += dS^T Q_i            tcgen05, A = dS^T (K-major), B = Q_i (MN-major)
-//   dQ_i  = dS K_j              tcgen05, A = dS^T read MN-major, B = K_j (MN-major)
+//   S'^T  = K_j Q_i^T  - 1 (LSE2_i / c)^T     tcgen05 (c = scale * log2 e)
+//   dP'^T = V_j dO_i^T - 1 D_i^T              tcgen05
+//   P^T   = 2^(c S'^T)      one thread per key row, masked, written back over
+//                           S'^T in TMEM as bf16
+//   dV_j += P^T dO_i        tcgen05, A = P^T (TMEM), B = dO_i (MN-major)
+//   dS^T  = P^T o dP'^T     written to shared memory as bf16
+//   dK_j += dS^T Q_i        tcgen05, A = dS^T (K-major), B = Q_i (MN-major)
+//   dQ_i  = dS K_j          tcgen05, A = dS^T read MN-major, B = K_j (MN-major)
+//
+// The per-query terms -LSE2_i / c and -D_i enter the two recompute GEMMs as
+// one extra K = 16 step: A is a constant slab whose first three columns are
+// 1, B a per-Q-tile slab holding the value split into three bf16 parts
+// (hi + mid + lo carries it to about fp32 accuracy).  The tensor core thus
+// does the per-column subtraction and the softmax threads load no per-column
+// values.  Warp 2 builds those slabs from LSE2 and D in global memory.
 //
 // Issue order of the tensor-core work: ... dV_i, S_{i+1}, dK_i, dQ_i, dP_{i+1},
 // dV_{i+1} ...  S_{i+1} goes right after dV_i (tcgen05.mma ops of one thread
@@ -27,11 +34,12 @@
 // are coalesced.
 //
 // Warp roles (384 threads): warp 0 TMA producer; warp 1 TMEM allocator and MMA
-// issuer; warps 4-7 compute P^T / dS^T (thread = key row) and write dK, dV;
-// warps 8-11 read dQ out of TMEM (thread = query row) and add it to global.
+// issuer; warp 2 builds the LSE / D slabs; warps 4-7 compute P^T / dS^T
+// (thread = key row) and write dK, dV; warps 8-11 read dQ out of TMEM
+// (thread = query row) and add it to global.
 //
-// TMEM columns:  dK [0,D), dV [D,2D), S^T/P^T [2D,2D+128), dP^T [2D+128,2D+256);
-// dQ reuses the dP^T columns once dS^T has been formed (d=128 fills all 512).
+// TMEM columns:  dK [0,D), dV [D,2D), S'^T/P^T [2D,2D+128), dP'^T [2D+128,2D+256);
+// dQ reuses the dP'^T columns once dS^T has been formed (d=128 fills all 512).
 #pragma once
 
 namespace fa {
@@ -39,27 +47,28 @@ namespace fa {
 template <int D>
 struct BwdLayout {
   static constexpr int kThreads = 384;
-  static constexpr int kTile = 128 * D * 2;  // bytes of a K, V, Q or dO tile
-  static constexpr int kSq = 128 * 128 * 2;  // bytes of the bf16 dS^T tile
+  static constexpr int kTile = 128 * D * 2;   // bytes of a K, V, Q or dO tile
+  static constexpr int kSq = 128 * 128 * 2;   // bytes of the bf16 dS^T tile
+  static constexpr int kSlab = 128 * 16 * 2;  // bytes of a 128 x 16 bf16 slab
+  static constexpr int kDoStages = (D == 64) ? 2 : 1;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTile;
-  static constexpr int kOffQ = kOffV + kTile;    // [2]
-  static constexpr int kOffDO = kOffQ + 2 * kTile;  // [2]
-  static constexpr int kOffDS = kOffDO + 2 * kTile;
-  static constexpr int kOffLse = kOffDS + kSq;  // [2] x 128 fp32 LSE (log2 units) of Q tile i
-  static constexpr int kOffDv = kOffLse + 1024;  // [2] x 128 fp32 D_i
-  static constexpr int kOffBar = kOffDv + 1024;
+  static constexpr int kOffQ = kOffV + kTile;                // [2]
+  static constexpr int kOffDO = kOffQ + 2 * kTile;           // [kDoStages]
+  static constexpr int kOffDS = kOffDO + kDoStages * kTile;
+  static constexpr int kOffOnes = kOffDS + kSq;              // constant A slab
+  static constexpr int kOffQSlab = kOffOnes + kSlab;         // [2] -LSE2/c parts
+  static constexpr int kOffDoSlab = kOffQSlab + 2 * kSlab;   // [kDoStages] -D parts
+  static constexpr int kOffBar = kOffDoSlab + kDoStages * kSlab;
   static constexpr int kBarArea = 256;
   static constexpr int kBytes = kOffBar + kBarArea;
-  // The 1 KiB alignment slack is kept only where it fits; without it the
-  // kernel checks that the dynamic shared memory base is 1 KiB aligned.
-  static constexpr int kSlack = (kBytes + 1024 <= 232448) ? 1024 : 0;
-  static constexpr int kSmemAlloc = kBytes + kSlack;
+  static constexpr int kSmemAlloc = kBytes + 1024;  // slack to align the base to 1 KiB
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   // barriers
-  static constexpr int kKvFull = 0, kQdoFull = 1 /*[2]*/, kQdoEmpty = 3 /*[2]*/, kSFull = 5,
-                       kPReady = 6, kDpFull = 7, kDsReady = 8, kDsFree = 9, kDqFull = 10,
-                       kDqFree = 11, kDkdvDone = 12, kDrain = 13, kNumBars = 14;
+  static constexpr int kKvFull = 0, kQFull = 1 /*[2]*/, kQEmpty = 3 /*[2]*/, kDoFull = 5 /*[2]*/,
+                       kDoEmpty = 7 /*[2]*/, kSFull = 9, kPReady = 10, kDpFull = 11,
+                       kDsReady = 12, kDsFree = 13, kDqFull = 14, kDqFree = 15, kDkdvDone = 16,
+                       kDrain = 17, kNumBars = 18;
   static constexpr int kOffSlot = kOffBar + 8 * kNumBars;
   static constexpr int kOffAbort = kOffSlot + 4;
   static_assert(kOffAbort + 4 <= kOffBar + kBarArea, "barrier area too small");
@@ -73,25 +82,50 @@ struct BwdLayout {
   static_assert(kColDP + 128 <= kTmemCols, "TMEM budget");
 };
 
+// Shared-memory descriptor of a 128 x 16 bf16 K-major slab with 32-byte
+// swizzle: row r at 32 r bytes, its two 16-byte halves swapped when bit 2 of r
+// is set; SBO = 256 bytes between 8-row groups; layout type 6.
+__device__ __forceinline__ uint64_t sw32_slab_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1) << 16;         // LBO (unused): 16 bytes
+  d |= static_cast<uint64_t>(256 >> 4) << 32;  // SBO
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(6) << 61;
+  return d;
+}
+
+// Writes row r of a slab: columns 0..2 hold v0, v1, v2 (bf16), the rest 0.
+__device__ __forceinline__ void slab_row(uint32_t slab, int r, float v0, float v1, float v2) {
+  const uint32_t lo = pack_bf16x2(v0, v1), hi = pack_bf16x2(v2, 0.f);
+  const uint32_t swz = static_cast<uint32_t>((r >> 2) & 1);
+  st_shared_v4(slab + r * 32 + (swz << 4), lo, hi, 0u, 0u);          // columns 0..7
+  st_shared_v4(slab + r * 32 + ((swz ^ 1u) << 4), 0u, 0u, 0u, 0u);  // columns 8..15
+}
+
+// x as three bf16-exact parts a + b + c (each part the bf16 rounding of the
+// remainder, so the sum matches x to about 2^-24 relative).
+__device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
+  a = __bfloat162float(__float2bfloat16_rn(x));
+  const float r1 = x - a;
+  b = __bfloat162float(__float2bfloat16_rn(r1));
+  c = __bfloat162float(__float2bfloat16_rn(r1 - b));
+}
+
 template <int D, bool kCausal>
 __global__ void __launch_bounds__(384, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                     const float* __restrict__ dvec, const float* __restrict__ lse2,
-                    float* __restrict__ dq_acc, int n, int np, float scale, float scale_log2,
+                    float* __restrict__ dq_acc, int n, int np, float scale, float c_exp,
                     uint64_t limit_ns) {
   using L = BwdLayout<D>;
   constexpr int kDBlk = D / 64;
+  constexpr int DS = L::kDoStages;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
-  if (L::kSlack == 0 && (raw_addr & 1023u) != 0) {
-    // every thread sees the same base: the whole CTA leaves before touching
-    // any barrier or TMEM
-    if (threadIdx.x == 0) atomicOr(&g_error_word, kErrBwdMain | kErrAlign);
-    return;
-  }
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + L::kOffBar + 8u * static_cast<uint32_t>(i); };
@@ -110,11 +144,16 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < L::kNumBars; ++b) {
       uint32_t cnt = 1;
-      if (b == L::kPReady || b == L::kDsReady || b == L::kDqFree) cnt = 4;
+      if (b == L::kPReady || b == L::kDsReady || b == L::kDqFree) cnt = 4;  // four warps
+      if ((b >= L::kQFull && b < L::kQFull + 2) || (b >= L::kDoFull && b < L::kDoFull + 2))
+        cnt = 2;  // the TMA producer and the slab builder
       mbar_init(bar(b), cnt);
     }
     *abort_flag = 0;
     fence_barrier_init();
+  }
+  if (threadIdx.x < 128) {  // constant A slab: 1 in the first three columns
+    slab_row(sb + L::kOffOnes, threadIdx.x, 1.f, 1.f, 1.f);
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -133,34 +172,41 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
+      const uint32_t err = err_k | kErrRoleLoad;
       mbar_arrive_expect_tx(bar(L::kKvFull), 2 * L::kTile);
       for (int db = 0; db < kDBlk; ++db) {
         tma_load_3d(sb + L::kOffK + db * 16384, &tm_k, bar(L::kKvFull), db * 64, j * 128, bh);
         tma_load_3d(sb + L::kOffV + db * 16384, &tm_v, bar(L::kKvFull), db * 64, j * 128, bh);
       }
-      int issued = 0;
+      int nq = 0, ndo = 0;
       for (int it = 0; it < n_it; ++it) {
         const int i = i0 + it;
         const int st = it & 1;
-        if (!wait_bounded(bar(L::kQdoEmpty + st), ((it >> 1) & 1) ^ 1, limit_ns, abort_flag,
-                          err_k | kErrRoleLoad))
+        if (!wait_bounded(bar(L::kQEmpty + st), ((it >> 1) & 1) ^ 1, limit_ns, abort_flag, err))
           break;
-        const uint32_t fb = bar(L::kQdoFull + st);
-        mbar_arrive_expect_tx(fb, 2 * L::kTile + 1024);
-        for (int db = 0; db < kDBlk; ++db) {
-          tma_load_3d(sb + L::kOffQ + st * L::kTile + db * 16384, &tm_q, fb, db * 64, i * 128, bh);
-          tma_load_3d(sb + L::kOffDO + st * L::kTile + db * 16384, &tm_do, fb, db * 64, i * 128,
-                      bh);
-        }
-        const size_t vrow = static_cast<size_t>(bh) * np + static_cast<size_t>(i) * 128;
-        bulk_load(sb + L::kOffLse + st * 512, lse2 + vrow, 512, fb);
-        bulk_load(sb + L::kOffDv + st * 512, dvec + vrow, 512, fb);
-        issued = it + 1;
+        mbar_arrive_expect_tx(bar(L::kQFull + st), L::kTile);
+        for (int db = 0; db < kDBlk; ++db)
+          tma_load_3d(sb + L::kOffQ + st * L::kTile + db * 16384, &tm_q, bar(L::kQFull + st),
+                      db * 64, i * 128, bh);
+        ++nq;
+        const int ds = it % DS;
+        if (!wait_bounded(bar(L::kDoEmpty + ds), ((it / DS) & 1) ^ 1, limit_ns, abort_flag, err))
+          break;
+        mbar_arrive_expect_tx(bar(L::kDoFull + ds), L::kTile);
+        for (int db = 0; db < kDBlk; ++db)
+          tma_load_3d(sb + L::kOffDO + ds * L::kTile + db * 16384, &tm_do, bar(L::kDoFull + ds),
+                      db * 64, i * 128, bh);
+        ++ndo;
       }
       if (*abort_flag) {
+        // copies already issued must land before shared memory is released;
+        // with the slab builder's arrival possibly missing, these waits may
+        // run to their limit, which only delays the exit
         drain_wait(bar(L::kKvFull), 0, limit_ns);
-        for (int it = (issued > 2 ? issued - 2 : 0); it < issued; ++it)
-          drain_wait(bar(L::kQdoFull + (it & 1)), (it >> 1) & 1, limit_ns);
+        for (int it = (nq > 2 ? nq - 2 : 0); it < nq; ++it)
+          drain_wait(bar(L::kQFull + (it & 1)), (it >> 1) & 1, limit_ns);
+        for (int it = (ndo > DS ? ndo - DS : 0); it < ndo; ++it)
+          drain_wait(bar(L::kDoFull + it % DS), (it / DS) & 1, limit_ns);
       }
     }
   } else if (warp == 1) {
@@ -171,7 +217,8 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t id_mnmn = idesc_bf16_f32(128, D, true, true);
       const uint32_t err = err_k | kErrRoleMma;
       const uint32_t a_k = sb + L::kOffK, a_v = sb + L::kOffV, a_ds = sb + L::kOffDS;
-      auto issue_s = [&](int it) {  // S^T = K_j Q_i^T
+      const uint64_t d_ones = sw32_slab_desc(sb + L::kOffOnes);
+      auto issue_s = [&](int it) {  // S'^T = K_j Q_i^T - 1 (LSE2_i / c)^T
         const uint32_t a_q = sb + L::kOffQ + (it & 1) * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -179,20 +226,26 @@ __global__ void __launch_bounds__(384, 1)
           mma_bf16_ss(tmem + L::kColS, sw128_desc(a_k + off, 16, 1024),
                       sw128_desc(a_q + off, 16, 1024), id_kk, kk > 0 ? 1u : 0u);
         }
+        mma_bf16_ss(tmem + L::kColS, d_ones,
+                    sw32_slab_desc(sb + L::kOffQSlab + (it & 1) * L::kSlab), id_kk, 1u);
         tc_commit(bar(L::kSFull));
       };
-      auto issue_dp = [&](int it) {  // dP^T = V_j dO_i^T
-        const uint32_t a_do = sb + L::kOffDO + (it & 1) * L::kTile;
+      auto issue_dp = [&](int it) {  // dP'^T = V_j dO_i^T - 1 D_i^T
+        const int ds = it % DS;
+        const uint32_t a_do = sb + L::kOffDO + ds * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
           mma_bf16_ss(tmem + L::kColDP, sw128_desc(a_v + off, 16, 1024),
                       sw128_desc(a_do + off, 16, 1024), id_kk, kk > 0 ? 1u : 0u);
         }
+        mma_bf16_ss(tmem + L::kColDP, d_ones,
+                    sw32_slab_desc(sb + L::kOffDoSlab + ds * L::kSlab), id_kk, 1u);
         tc_commit(bar(L::kDpFull));
       };
       bool ok = wait_bounded(bar(L::kKvFull), 0, limit_ns, abort_flag, err) &&
-                wait_bounded(bar(L::kQdoFull), 0, limit_ns, abort_flag, err);
+                wait_bounded(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
+                wait_bounded(bar(L::kDoFull), 0, limit_ns, abort_flag, err);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -201,8 +254,9 @@ __global__ void __launch_bounds__(384, 1)
       for (int it = 0; ok && it < n_it; ++it) {
         const uint32_t ph = it & 1;
         const int st = it & 1;
+        const int ds = it % DS;
         const uint32_t a_q = sb + L::kOffQ + st * L::kTile;
-        const uint32_t a_do = sb + L::kOffDO + st * L::kTile;
+        const uint32_t a_do = sb + L::kOffDO + ds * L::kTile;
         const bool next = it + 1 < n_it;
         if (!wait_bounded(bar(L::kPReady), ph, limit_ns, abort_flag, err)) break;
         tc_fence_after();
@@ -211,8 +265,9 @@ __global__ void __launch_bounds__(384, 1)
           mma_bf16_ts(tmem + L::kColDV, tmem + L::kColS + kk * 8,
                       sw128_desc(a_do + kk * 2048, 16384, 1024), id_kmn,
                       (it > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(L::kDoEmpty + ds));  // dO_i and its slab are no longer read
         if (next) {  // S of the next Q tile, as soon as P_i has been consumed
-          if (!wait_bounded(bar(L::kQdoFull + ((it + 1) & 1)), ((it + 1) >> 1) & 1, limit_ns,
+          if (!wait_bounded(bar(L::kQFull + ((it + 1) & 1)), ((it + 1) >> 1) & 1, limit_ns,
                             abort_flag, err))
             break;
           tc_fence_after();
@@ -227,7 +282,7 @@ __global__ void __launch_bounds__(384, 1)
                       sw128_desc(a_q + kk * 2048, 16384, 1024), id_kmn,
                       (it > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(L::kQdoEmpty + st));  // Q_i, dO_i, LSE_i, D_i no longer read
+        tc_commit(bar(L::kQEmpty + st));  // Q_i and its slab are no longer read
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dQ_i = dS K_j  (K = 128 keys)
           mma_bf16_ss(tmem + L::kColDQ, sw128_desc(a_ds + kk * 2048, 16384, 1024),
@@ -236,6 +291,9 @@ __global__ void __launch_bounds__(384, 1)
         tc_commit(bar(L::kDsFree));
         if (next) {  // dP of the next Q tile once dQ_i has left the shared columns
           if (!wait_bounded(bar(L::kDqFree), ph, limit_ns, abort_flag, err)) break;
+          if (!wait_bounded(bar(L::kDoFull + (it + 1) % DS), ((it + 1) / DS) & 1, limit_ns,
+                            abort_flag, err))
+            break;
           tc_fence_after();
           issue_dp(it + 1);
         }
@@ -245,6 +303,50 @@ __global__ void __launch_bounds__(384, 1)
       drain_wait(bar(L::kDrain), 0, limit_ns);
     }
     __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------- slab builder
+    // Q slab of tile i: row q holds -LSE2_q / c in three bf16 parts; dO slab:
+    // -D_q in three parts.  Rows past the end of the sequence (LSE2 = +inf)
+    // get a large finite value whose scaled exponential is 0.
+    const uint32_t err = err_k | kErrRoleLoad;
+    const float inv_c = 1.0f / c_exp;
+    // c * pad = -200 (or beyond): its base-2 exponential is 0 in fp32
+    const float pad = copysignf(fminf(200.0f / fabsf(c_exp), 3.0e38f), -c_exp);
+    for (int it = 0; it < n_it; ++it) {
+      const int i = i0 + it;
+      const int st = it & 1;
+      const size_t vrow =
+          static_cast<size_t>(bh) * np + static_cast<size_t>(i) * 128 + static_cast<size_t>(lane) * 4;
+      const float4 l4 = *reinterpret_cast<const float4*>(lse2 + vrow);
+      const float4 d4 = *reinterpret_cast<const float4*>(dvec + vrow);
+      if (!wait_bounded_warp(bar(L::kQEmpty + st), ((it >> 1) & 1) ^ 1, limit_ns, abort_flag, err))
+        break;
+      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x = (lv[e] == INFINITY) ? pad : -lv[e] * inv_c;
+        float a, b, c;
+        split3(x, a, b, c);
+        slab_row(sb + L::kOffQSlab + st * L::kSlab, lane * 4 + e, a, b, c);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kQFull + st));
+      const int ds = it % DS;
+      if (!wait_bounded_warp(bar(L::kDoEmpty + ds), ((it / DS) & 1) ^ 1, limit_ns, abort_flag,
+                             err))
+        break;
+      const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float a, b, c;
+        split3(-dv[e], a, b, c);
+        slab_row(sb + L::kOffDoSlab + ds * L::kSlab, lane * 4 + e, a, b, c);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kDoFull + ds));
+    }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------ P^T, dS^T, dK / dV out
     const int r = threadIdx.x - 128;  // key row in the tile == TMEM lane
@@ -257,11 +359,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int it = 0; it < n_it; ++it) {
       const int i = i0 + it;
       const uint32_t ph = it & 1;
-      const int st = it & 1;
-      const float4* lse4 = reinterpret_cast<const float4*>(smem + L::kOffLse + st * 512);
-      const float4* d4 = reinterpret_cast<const float4*>(smem + L::kOffDv + st * 512);
-      if (!wait_bounded_warp(bar(L::kQdoFull + st), (it >> 1) & 1, limit_ns, abort_flag, err) ||
-          !wait_bounded_warp(bar(L::kSFull), ph, limit_ns, abort_flag, err)) {
+      if (!wait_bounded_warp(bar(L::kSFull), ph, limit_ns, abort_flag, err)) {
         ok = false;
         break;
       }
@@ -277,25 +375,19 @@ __global__ void __launch_bounds__(384, 1)
                            *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
         tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 l = lse4[h * 16 + c4];
-          const int c = h * 64 + c4 * 4;
-          float p0 = ex2_approx(fmaf(__uint_as_float(u[c4 * 4 + 0]), scale_log2, -l.x));
-          float p1 = ex2_approx(fmaf(__uint_as_float(u[c4 * 4 + 1]), scale_log2, -l.y));
-          float p2 = ex2_approx(fmaf(__uint_as_float(u[c4 * 4 + 2]), scale_log2, -l.z));
-          float p3 = ex2_approx(fmaf(__uint_as_float(u[c4 * 4 + 3]), scale_log2, -l.w));
+        for (int e = 0; e < 64; e += 2) {
+          const int c = h * 64 + e;
+          float p0 = ex2_approx(__uint_as_float(u[e]) * c_exp);
+          float p1 = ex2_approx(__uint_as_float(u[e + 1]) * c_exp);
           if (diag) {  // keep key r for query c iff r <= c
-            p0 = (c + 0 >= r) ? p0 : 0.f;
+            p0 = (c >= r) ? p0 : 0.f;
             p1 = (c + 1 >= r) ? p1 : 0.f;
-            p2 = (c + 2 >= r) ? p2 : 0.f;
-            p3 = (c + 3 >= r) ? p3 : 0.f;
           }
-          if (!key_ok) p0 = p1 = p2 = p3 = 0.f;
+          if (!key_ok) p0 = p1 = 0.f;
           pk[c / 2] = pack_bf16x2(p0, p1);
-          pk[c / 2 + 1] = pack_bf16x2(p2, p3);
         }
-        // P^T over the first 64 TMEM columns of S^T (bf16 pairs): this half's
-        // 32 packed columns land on S^T columns already read
+        // P^T over the first 64 TMEM columns of S'^T (bf16 pairs): this half's
+        // 32 packed columns land on columns already read
         tmem_st_32x32b_x32(tmem + lane_off + L::kColS + h * 32,
                            *reinterpret_cast<const uint32_t(*)[32]>(&pk[h * 32]));
       }
@@ -318,16 +410,10 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const int c = cc * 32 + e;
-          const float4 dd = d4[c / 4];
-          const uint32_t pa = pk[c / 2], pb = pk[c / 2 + 1];
-          const float s0 = bf16_lo(pa) * (__uint_as_float(u[e + 0]) - dd.x);
-          const float s1 = bf16_hi(pa) * (__uint_as_float(u[e + 1]) - dd.y);
-          const float s2 = bf16_lo(pb) * (__uint_as_float(u[e + 2]) - dd.z);
-          const float s3 = bf16_hi(pb) * (__uint_as_float(u[e + 3]) - dd.w);
-          w[e / 2] = pack_bf16x2(s0, s1);
-          w[e / 2 + 1] = pack_bf16x2(s2, s3);
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t pp = pk[(cc * 32 + e) / 2];
+          w[e / 2] = pack_bf16x2(bf16_lo(pp) * __uint_as_float(u[e]),
+                                 bf16_hi(pp) * __uint_as_float(u[e + 1]));
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {

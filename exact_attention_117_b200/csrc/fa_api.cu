@@ -183,6 +183,11 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   }
   const int np = static_cast<int>(round_up(static_cast<size_t>(N), 128));
   const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  // exponent factor of the main kernel: it subtracts LSE2 / c inside the score
+  // GEMM, so c must not be 0; below 1e-30 every scaled score is 0 to fp32
+  // accuracy anyway, and the exact scale is applied to dQ and dK afterwards
+  const float c_exp = std::fabs(scale_log2) < 1e-30f ? (scale_log2 < 0.f ? -1e-30f : 1e-30f)
+                                                     : scale_log2;
   {
     LaunchTimer timer(st, FA_KERNEL_BWD_PRE);
     const long long rows = static_cast<long long>(BH) * np;
@@ -196,7 +201,7 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     LaunchTimer timer(st, FA_KERNEL_BWD_MAIN);
     dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(np / 128));
     fa::bwd_main_kernel<D, C><<<grid, L::kThreads, L::kSmemAlloc, st>>>(
-        mq, mk, mv, mdo, mdk, mdv, ws.dvec, ws.lse2, ws.dq_acc, N, np, scale, scale_log2,
+        mq, mk, mv, mdo, mdk, mdv, ws.dvec, ws.lse2, ws.dq_acc, N, np, scale, c_exp,
         kWaitLimitNs);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
