@@ -70,10 +70,12 @@ __global__ void __launch_bounds__(256)
     // rows past the end get +inf so that their recomputed probabilities are 0
     lse2[vrow] = (r < n) ? lse[static_cast<size_t>(bh) * n + r] * log2e : INFINITY;
   }
-  float4* acc_row = reinterpret_cast<float4*>(dq_acc + vrow * D);
-  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (dq_acc != nullptr) {  // the deterministic backward has no accumulator
+    float4* acc_row = reinterpret_cast<float4*>(dq_acc + vrow * D);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int i = lane; i < D / 4; i += 32) acc_row[i] = z;
+    for (int i = lane; i < D / 4; i += 32) acc_row[i] = z;
+  }
 }
 
 // ------------------------------------------------------------- dQ convert
@@ -105,3 +107,4 @@ __global__ void __launch_bounds__(256)
 }  // namespace fa
 
 #include "bwd_main.cuh"
+#include "dq_pass.cuh"

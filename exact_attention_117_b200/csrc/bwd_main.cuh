@@ -36,7 +36,10 @@
 // Warp roles (384 threads): warp 0 TMA producer; warp 1 TMEM allocator and MMA
 // issuer; warp 2 builds the LSE / D slabs; warps 4-7 compute P^T / dS^T
 // (thread = key row) and write dK, dV; warps 8-11 read dQ out of TMEM
-// (thread = query row) and add it to global.
+// (thread = query row) and add it to global.  Without dQ (the deterministic
+// backward) warps 8-11 instead share the P^T / dS^T work: each warp group
+// takes 64 of the 128 query columns.  P^T of query half h sits in the first
+// 32 of the 64 TMEM columns S'^T had for those queries.
 //
 // TMEM columns:  dK [0,D), dV [D,2D), S'^T/P^T [2D,2D+128), dP'^T [2D+128,2D+256);
 // dQ reuses the dP'^T columns once dS^T has been formed (d=128 fills all 512).
@@ -112,7 +115,9 @@ __device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
   c = __bfloat162float(__float2bfloat16_rn(r1 - b));
 }
 
-template <int D, bool kCausal>
+// kDq = false (deterministic backward): no dQ MMA and no atomics here; dQ
+// comes from dq_pass_kernel.  dP_{i+1} then only waits for dS_i to be formed.
+template <int D, bool kCausal, bool kDq>
 __global__ void __launch_bounds__(384, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -144,7 +149,8 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < L::kNumBars; ++b) {
       uint32_t cnt = 1;
-      if (b == L::kPReady || b == L::kDsReady || b == L::kDqFree) cnt = 4;  // four warps
+      if (b == L::kDqFree) cnt = 4;  // the dQ read-out warps
+      if (b == L::kPReady || b == L::kDsReady) cnt = kDq ? 4 : 8;  // the compute warps
       if ((b >= L::kQFull && b < L::kQFull + 2) || (b >= L::kDoFull && b < L::kDoFull + 2))
         cnt = 2;  // the TMA producer and the slab builder
       mbar_init(bar(b), cnt);
@@ -262,7 +268,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dV_j += P^T dO_i  (K = 128 queries, P^T in TMEM)
-          mma_bf16_ts(tmem + L::kColDV, tmem + L::kColS + kk * 8,
+          mma_bf16_ts(tmem + L::kColDV, tmem + L::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
                       sw128_desc(a_do + kk * 2048, 16384, 1024), id_kmn,
                       (it > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(L::kDoEmpty + ds));  // dO_i and its slab are no longer read
@@ -283,14 +289,16 @@ __global__ void __launch_bounds__(384, 1)
                       (it > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar(L::kQEmpty + st));  // Q_i and its slab are no longer read
+        if (kDq) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // dQ_i = dS K_j  (K = 128 keys)
-          mma_bf16_ss(tmem + L::kColDQ, sw128_desc(a_ds + kk * 2048, 16384, 1024),
-                      sw128_desc(a_k + kk * 2048, 16384, 1024), id_mnmn, kk > 0 ? 1u : 0u);
-        tc_commit(bar(L::kDqFull));
+          for (int kk = 0; kk < 8; ++kk)  // dQ_i = dS K_j  (K = 128 keys)
+            mma_bf16_ss(tmem + L::kColDQ, sw128_desc(a_ds + kk * 2048, 16384, 1024),
+                        sw128_desc(a_k + kk * 2048, 16384, 1024), id_mnmn, kk > 0 ? 1u : 0u);
+          tc_commit(bar(L::kDqFull));
+        }
         tc_commit(bar(L::kDsFree));
         if (next) {  // dP of the next Q tile once dQ_i has left the shared columns
-          if (!wait_bounded(bar(L::kDqFree), ph, limit_ns, abort_flag, err)) break;
+          if (kDq && !wait_bounded(bar(L::kDqFree), ph, limit_ns, abort_flag, err)) break;
           if (!wait_bounded(bar(L::kDoFull + (it + 1) % DS), ((it + 1) / DS) & 1, limit_ns,
                             abort_flag, err))
             break;
@@ -347,9 +355,14 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::kDoFull + ds));
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && (warp < 8 || !kDq)) {
     // ------------------------------------------------ P^T, dS^T, dK / dV out
-    const int r = threadIdx.x - 128;  // key row in the tile == TMEM lane
+    // kDq: warps 4-7 take all 128 query columns; otherwise warps 4-7 take
+    // queries 0-63 and warps 8-11 queries 64-127 (and the two halves of dK, dV)
+    constexpr int kHalves = kDq ? 2 : 1;
+    constexpr int kWgThreads = kDq ? 128 : 256;
+    const int h0 = kDq ? 0 : (warp >> 2) - 1;
+    const int r = (warp & 3) * 32 + lane;  // key row in the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int key = j * 128 + r;
     const bool key_ok = key < n;
@@ -365,9 +378,10 @@ __global__ void __launch_bounds__(384, 1)
       }
       tc_fence_after();
       const bool diag = kCausal && (i == j);
-      uint32_t pk[64];  // P^T row as bf16 pairs, kept for dS
+      uint32_t pk[32 * kHalves];  // P^T row as bf16 pairs, kept for dS
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {  // two halves of 64 query columns
+      for (int hh = 0; hh < kHalves; ++hh) {  // halves of 64 query columns
+        const int h = h0 + hh;
         uint32_t u[64];
         tmem_ld_32x32b_x32(tmem + lane_off + L::kColS + h * 64,
                            *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
@@ -384,12 +398,12 @@ __global__ void __launch_bounds__(384, 1)
             p1 = (c + 1 >= r) ? p1 : 0.f;
           }
           if (!key_ok) p0 = p1 = 0.f;
-          pk[c / 2] = pack_bf16x2(p0, p1);
+          pk[hh * 32 + e / 2] = pack_bf16x2(p0, p1);
         }
-        // P^T over the first 64 TMEM columns of S'^T (bf16 pairs): this half's
-        // 32 packed columns land on columns already read
-        tmem_st_32x32b_x32(tmem + lane_off + L::kColS + h * 32,
-                           *reinterpret_cast<const uint32_t(*)[32]>(&pk[h * 32]));
+        // P^T of this half over the first 32 of its own 64 TMEM columns of
+        // S'^T (bf16 pairs), which have been read
+        tmem_st_32x32b_x32(tmem + lane_off + L::kColS + h * 64,
+                           *reinterpret_cast<const uint32_t(*)[32]>(&pk[hh * 32]));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -404,14 +418,15 @@ __global__ void __launch_bounds__(384, 1)
       }
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {  // 32 query columns at a time
+      for (int cl = 0; cl < 2 * kHalves; ++cl) {  // 32 query columns at a time
+        const int cc = 2 * h0 + cl;
         uint32_t u[32];
         tmem_ld_32x32b_x32(tmem + lane_off + L::kColDP + cc * 32, u);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const uint32_t pp = pk[(cc * 32 + e) / 2];
+          const uint32_t pp = pk[(cl * 32 + e) / 2];
           w[e / 2] = pack_bf16x2(bf16_lo(pp) * __uint_as_float(u[e]),
                                  bf16_hi(pp) * __uint_as_float(u[e + 1]));
         }
@@ -431,6 +446,8 @@ __global__ void __launch_bounds__(384, 1)
     // dK (scaled) then dV go through the dS^T tile (free once every MMA is
     // done) as bf16 128-byte-swizzled rows, stored with TMA (rows >= N clip).
     if (ok) ok = wait_bounded_warp(bar(L::kDkdvDone), 0, limit_ns, abort_flag, err_k | kErrRoleEpilogue);
+    constexpr int kCols = D / 32 / (kDq ? 1 : 2);  // 32-column loads per thread
+    const int c_first = kDq ? 0 : h0 * kCols;
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
       if (ok) {
@@ -439,7 +456,8 @@ __global__ void __launch_bounds__(384, 1)
         const float mul = which == 0 ? scale : 1.0f;
         const uint32_t orow = sb + L::kOffDS + r * 128;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int cl = 0; cl < kCols; ++cl) {
+          const int c = c_first + cl;
           uint32_t u[32];
           tmem_ld_32x32b_x32(tmem + lane_off + col + c * 32, u);
           tmem_wait_ld();
@@ -460,17 +478,17 @@ __global__ void __launch_bounds__(384, 1)
         fence_proxy_async_smem();
       }
       tc_fence_before();
-      named_barrier_sync(1, 128);  // all four warps, ok or not
-      if (r == 0 && ok && !*abort_flag) {
+      named_barrier_sync(1, kWgThreads);  // all compute warps, ok or not
+      if (threadIdx.x == 128 && ok && !*abort_flag) {
         const CUtensorMap* map = which == 0 ? &tm_dk : &tm_dv;
         for (int db = 0; db < kDBlk; ++db)
           tma_store_3d(map, sb + L::kOffDS + db * 16384, db * 64, j * 128, bh);
         bulk_commit_group();
         bulk_wait_group_0();  // the staging tile is reused for dV
       }
-      named_barrier_sync(1, 128);
+      named_barrier_sync(1, kWgThreads);
     }
-  } else if (warp >= 8) {
+  } else if (kDq && warp >= 8) {
     // --------------------------------------------------------- dQ read-out
     const int c = threadIdx.x - 256;  // query row in the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;

@@ -18,6 +18,7 @@ enum : unsigned int {
   kErrFwd = 1u << 0,
   kErrBwdMain = 1u << 1,
   kErrBwdPre = 1u << 2,
+  kErrBwdDq = 1u << 3,
   kErrRoleLoad = 1u << 8,
   kErrRoleMma = 1u << 9,
   kErrRoleSoftmax = 1u << 10,

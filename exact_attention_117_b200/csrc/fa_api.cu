@@ -168,17 +168,20 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool C>
+template <int D, bool C, bool kDet>
 fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
-                     const void* o, const void* dout, const float* lse, void* dq,
-                     const BwdWorkspace& ws, int BH, int N, float scale, cudaStream_t st) {
+                     const CUtensorMap& mdq, const void* o, const void* dout, const float* lse,
+                     void* dq, const BwdWorkspace& ws, int BH, int N, float scale,
+                     cudaStream_t st) {
   using L = fa::BwdLayout<D>;
+  using LQ = fa::DqLayout<D>;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return FA_ERR_CUDA;
   if (!attr_set[dev]) {
-    if (!set_smem(fa::bwd_main_kernel<D, C>, L::kSmemAlloc)) return FA_ERR_CUDA;
+    if (!set_smem(fa::bwd_main_kernel<D, C, !kDet>, L::kSmemAlloc)) return FA_ERR_CUDA;
+    if (kDet && !set_smem(fa::dq_pass_kernel<D, C>, LQ::kSmemAlloc)) return FA_ERR_CUDA;
     attr_set[dev] = true;
   }
   const int np = static_cast<int>(round_up(static_cast<size_t>(N), 128));
@@ -194,18 +197,24 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);  // 8 rows (warps) per block
     fa::bwd_preprocess_kernel<D><<<blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
-        ws.dvec, ws.lse2, ws.dq_acc, BH, N, np, static_cast<float>(1.4426950408889634));
+        ws.dvec, ws.lse2, kDet ? nullptr : ws.dq_acc, BH, N, np,
+        static_cast<float>(1.4426950408889634));
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   {
     LaunchTimer timer(st, FA_KERNEL_BWD_MAIN);
     dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(np / 128));
-    fa::bwd_main_kernel<D, C><<<grid, L::kThreads, L::kSmemAlloc, st>>>(
+    fa::bwd_main_kernel<D, C, !kDet><<<grid, L::kThreads, L::kSmemAlloc, st>>>(
         mq, mk, mv, mdo, mdk, mdv, ws.dvec, ws.lse2, ws.dq_acc, N, np, scale, c_exp,
         kWaitLimitNs);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  {
+  if (kDet) {
+    LaunchTimer timer(st, FA_KERNEL_BWD_DQ);
+    dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(np / 128));
+    fa::dq_pass_kernel<D, C><<<grid, LQ::kThreads, LQ::kSmemAlloc, st>>>(
+        mq, mk, mv, mdo, mdq, ws.dvec, ws.lse2, N, np, scale, scale_log2, kWaitLimitNs);
+  } else {
     LaunchTimer timer(st, FA_KERNEL_BWD_DQ);
     const long long elems = static_cast<long long>(BH) * N * D;
     const unsigned blocks = static_cast<unsigned>((elems / 8 + 255) / 256);
@@ -213,6 +222,42 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
                                                       BH, N, np, scale);
   }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Shared body of fa_bwd and fa_bwd_deterministic.
+template <bool kDet>
+fa_status bwd_entry(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                    size_t workspace_bytes, int B, int H, int N, int d, int causal, float scale,
+                    void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGN;
+  const size_t need = bwd_workspace_layout(nullptr, B, H, N, d).bytes;
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGN;
+  const int bh = B * H;
+  BwdWorkspace ws = bwd_workspace_layout(workspace, B, H, N, d);
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
+  if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
+      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mdo, dout, d, N, bh, 128) ||
+      !encode_bf16_3d(&mdk, dk, d, N, bh, 128) || !encode_bf16_3d(&mdv, dv, d, N, bh, 128) ||
+      !encode_bf16_3d(&mdq, dq, d, N, bh, 128))
+    return FA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return causal ? launch_bwd<64, true, kDet>(mq, mk, mv, mdo, mdk, mdv, mdq, o, dout, lse, dq,
+                                               ws, bh, N, scale, s)
+                  : launch_bwd<64, false, kDet>(mq, mk, mv, mdo, mdk, mdv, mdq, o, dout, lse, dq,
+                                                ws, bh, N, scale, s);
+  return causal ? launch_bwd<128, true, kDet>(mq, mk, mv, mdo, mdk, mdv, mdq, o, dout, lse, dq,
+                                              ws, bh, N, scale, s)
+                : launch_bwd<128, false, kDet>(mq, mk, mv, mdo, mdk, mdv, mdq, o, dout, lse, dq,
+                                               ws, bh, N, scale, s);
 }
 
 }  // namespace
@@ -306,33 +351,16 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  const void* dout, void* dq, void* dk, void* dv, void* workspace,
                  size_t workspace_bytes, int B, int H, int N, int d, int causal, float scale,
                  void* stream) {
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_NULL;
-  fa_status st = check_common(B, H, N, d, scale);
-  if (st != FA_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return FA_ERR_ALIGN;
-  const size_t need = bwd_workspace_layout(nullptr, B, H, N, d).bytes;
-  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return FA_ERR_ALIGN;
-  const int bh = B * H;
-  BwdWorkspace ws = bwd_workspace_layout(workspace, B, H, N, d);
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
-  if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
-      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mdo, dout, d, N, bh, 128) ||
-      !encode_bf16_3d(&mdk, dk, d, N, bh, 128) || !encode_bf16_3d(&mdv, dv, d, N, bh, 128))
-    return FA_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64)
-    return causal ? launch_bwd<64, true>(mq, mk, mv, mdo, mdk, mdv, o, dout, lse, dq, ws, bh, N,
-                                         scale, s)
-                  : launch_bwd<64, false>(mq, mk, mv, mdo, mdk, mdv, o, dout, lse, dq, ws, bh, N,
-                                          scale, s);
-  return causal ? launch_bwd<128, true>(mq, mk, mv, mdo, mdk, mdv, o, dout, lse, dq, ws, bh, N,
-                                        scale, s)
-                : launch_bwd<128, false>(mq, mk, mv, mdo, mdk, mdv, o, dout, lse, dq, ws, bh, N,
-                                         scale, s);
+  return bwd_entry<false>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, N,
+                          d, causal, scale, stream);
+}
+
+fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                               const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                               void* workspace, size_t workspace_bytes, int B, int H, int N,
+                               int d, int causal, float scale, void* stream) {
+  return bwd_entry<true>(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, N,
+                         d, causal, scale, stream);
 }
 
 }  // extern "C"

@@ -56,6 +56,8 @@ def load() -> ctypes.CDLL:
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd.restype = i
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, vp]
+    lib.fa_bwd_deterministic.restype = i
+    lib.fa_bwd_deterministic.argtypes = lib.fa_bwd.argtypes
     lib.fa_bwd_noalloc.restype = i
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
     lib.fa_check_device_error.restype = i
@@ -157,9 +159,20 @@ def forward_splitkv(q, k, v, causal: bool = False, scale: Optional[float] = None
     return out, lse
 
 
+def bwd_deterministic_raw(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, H, N, d, causal,
+                          scale, stream) -> int:
+    """Direct call of ``fa_bwd_deterministic`` with raw pointers; returns the status code."""
+    return load().fa_bwd_deterministic(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, H, N, d,
+                                       int(bool(causal)), float(scale), stream)
+
+
 def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None,
-             dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """dQ, dK, dV of sum(dO * O); the fp32 workspace is allocated here if not given."""
+             dq=None, dk=None, dv=None, workspace=None, stream=None,
+             deterministic: bool = False):
+    """dQ, dK, dV of sum(dO * O); the fp32 workspace is allocated here if not given.
+
+    ``deterministic=True`` calls ``fa_bwd_deterministic`` (dQ summed in a fixed
+    order, bitwise reproducible) instead of ``fa_bwd`` (dQ summed by atomics)."""
     _check_qkv(q, k, v, o, do)
     B, H, N, d = q.shape
     if scale is None:
@@ -172,9 +185,11 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] =
     need = workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    _check(bwd_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
-                   _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                   B, H, N, d, causal, scale, _stream_ptr(stream)), "fa_bwd")
+    raw, name = (bwd_deterministic_raw, "fa_bwd_deterministic") if deterministic else \
+        (bwd_raw, "fa_bwd")
+    _check(raw(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+               _ptr(dv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+               B, H, N, d, causal, scale, _stream_ptr(stream)), name)
     return dq, dk, dv
 
 

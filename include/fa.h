@@ -129,6 +129,27 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  int B, int H, int N, int d, int causal, float scale, void* stream);
 
 /*
+ * Deterministic backward: same arguments, workspace size, preconditions and
+ * results as fa_bwd, but dQ is bitwise reproducible from run to run.
+ *
+ * Same recompute backward ("从零实现 FlashAttention-2：分块在线 Softmax",
+ * section 反向传播：重算，而不是存储), with the work split in two passes so that
+ * no output is summed by atomics: a key-tile-owned pass writes dK and dV
+ * exactly as fa_bwd does, and a query-tile-owned pass recomputes the score
+ * and dP tiles of each 128-row query tile against every key tile it sees,
+ * summing dQ = scale * sum_j dS_j K_j in one fixed order in on-chip
+ * accumulators and writing it once.  Costs one extra recompute of S and dP
+ * (7 instead of 5 tile GEMMs per tile pair).  Only the two fp32 row vectors
+ * of the workspace are used.
+ */
+FA_API fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v,
+                                      const void* o, const float* lse, const void* dout,
+                                      void* dq, void* dk, void* dv,
+                                      void* workspace, size_t workspace_bytes,
+                                      int B, int H, int N, int d, int causal, float scale,
+                                      void* stream);
+
+/*
  * Backward pass that allocates nothing.  (The pages have no counterpart to
  * this entry point: it exists only for callers that cannot allocate.)
  *

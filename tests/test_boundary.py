@@ -48,12 +48,12 @@ def _fwd(lib, q=P, k=P, v=P, o=P, lse=P, B=1, H=1, N=128, d=64, causal=0, scale=
     return fa.fwd_raw(q, k, v, o, lse, B, H, N, d, causal, scale, 0)
 
 
-def _bwd(lib, ptrs=None, ws=P, ws_bytes=None, B=1, H=1, N=128, d=64, scale=0.125):
+def _bwd(lib, ptrs=None, ws=P, ws_bytes=None, B=1, H=1, N=128, d=64, scale=0.125, raw=None):
     from exact_attention_117_b200 import fa
     p = ptrs or [P] * 9
     if ws_bytes is None:
         ws_bytes = fa.workspace_size(B, H, N, d) if d in (64, 128) and N > 0 else 1 << 20
-    return fa.bwd_raw(*p[:6], *p[6:9], ws, ws_bytes, B, H, N, d, 0, scale, 0)
+    return (raw or fa.bwd_raw)(*p[:6], *p[6:9], ws, ws_bytes, B, H, N, d, 0, scale, 0)
 
 
 def test_fwd_rejects_null(lib):
@@ -84,21 +84,23 @@ def test_fwd_rejects_scale(lib, scale):
     assert _fwd(lib, scale=scale) == 5
 
 
-def test_bwd_checks(lib):
+@pytest.mark.parametrize("entry", ["bwd_raw", "bwd_deterministic_raw"])
+def test_bwd_checks(lib, entry):
     from exact_attention_117_b200 import fa
+    raw = getattr(fa, entry)
     for i in range(9):
         p = [P] * 9
         p[i] = None
-        assert _bwd(lib, ptrs=p) == 1
-    assert _bwd(lib, N=0) == 2
-    assert _bwd(lib, d=80) == 3
+        assert _bwd(lib, ptrs=p, raw=raw) == 1
+    assert _bwd(lib, N=0, raw=raw) == 2
+    assert _bwd(lib, d=80, raw=raw) == 3
     p = [P] * 9
     p[7] = P + 4
-    assert _bwd(lib, ptrs=p) == 4
-    assert _bwd(lib, scale=math.nan) == 5
+    assert _bwd(lib, ptrs=p, raw=raw) == 4
+    assert _bwd(lib, scale=math.nan, raw=raw) == 5
     need = fa.workspace_size(1, 1, 128, 64)
-    assert _bwd(lib, ws=None) == 6
-    assert _bwd(lib, ws_bytes=need - 1) == 6
+    assert _bwd(lib, ws=None, raw=raw) == 6
+    assert _bwd(lib, ws_bytes=need - 1, raw=raw) == 6
 
 
 def test_workspace_size(lib):
