@@ -217,7 +217,8 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // the whole warp runs this loop; the MMA and commit wrappers elect one lane
+    {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t id_kmn = idesc_bf16_f32(128, D, false, true);
       constexpr uint32_t id_mnmn = idesc_bf16_f32(128, D, true, true);
@@ -249,9 +250,9 @@ __global__ void __launch_bounds__(384, 1)
                     sw32_slab_desc(sb + L::kOffDoSlab + ds * L::kSlab), id_kk, 1u);
         tc_commit(bar(L::kDpFull));
       };
-      bool ok = wait_bounded(bar(L::kKvFull), 0, limit_ns, abort_flag, err) &&
-                wait_bounded(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
-                wait_bounded(bar(L::kDoFull), 0, limit_ns, abort_flag, err);
+      bool ok = wait_bounded_warp(bar(L::kKvFull), 0, limit_ns, abort_flag, err) &&
+                wait_bounded_warp(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
+                wait_bounded_warp(bar(L::kDoFull), 0, limit_ns, abort_flag, err);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t a_q = sb + L::kOffQ + st * L::kTile;
         const uint32_t a_do = sb + L::kOffDO + ds * L::kTile;
         const bool next = it + 1 < n_it;
-        if (!wait_bounded(bar(L::kPReady), ph, limit_ns, abort_flag, err)) break;
+        if (!wait_bounded_warp(bar(L::kPReady), ph, limit_ns, abort_flag, err)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)  // dV_j += P^T dO_i  (K = 128 queries, P^T in TMEM)
@@ -273,20 +274,25 @@ __global__ void __launch_bounds__(384, 1)
                       (it > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(L::kDoEmpty + ds));  // dO_i and its slab are no longer read
         if (next) {  // S of the next Q tile, as soon as P_i has been consumed
-          if (!wait_bounded(bar(L::kQFull + ((it + 1) & 1)), ((it + 1) >> 1) & 1, limit_ns,
+          if (!wait_bounded_warp(bar(L::kQFull + ((it + 1) & 1)), ((it + 1) >> 1) & 1, limit_ns,
                             abort_flag, err))
             break;
           tc_fence_after();
           issue_s(it + 1);
         }
-        if (!wait_bounded(bar(L::kDsReady), ph, limit_ns, abort_flag, err)) break;
+        if (!wait_bounded_warp(bar(L::kDsReady), ph, limit_ns, abort_flag, err)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dK_j += dS^T Q_i
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + L::kColDK, sw128_desc(a_ds + off, 16, 1024),
-                      sw128_desc(a_q + kk * 2048, 16384, 1024), id_kmn,
-                      (it > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          if (kDq) {  // dS^T from shared memory (K-major)
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_bf16_ss(tmem + L::kColDK, sw128_desc(a_ds + off, 16, 1024),
+                        sw128_desc(a_q + kk * 2048, 16384, 1024), id_kmn, acc);
+          } else {  // dS^T from TMEM over dP'^T, laid out like P^T
+            mma_bf16_ts(tmem + L::kColDK, tmem + L::kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
+                        sw128_desc(a_q + kk * 2048, 16384, 1024), id_kmn, acc);
+          }
         }
         tc_commit(bar(L::kQEmpty + st));  // Q_i and its slab are no longer read
         if (kDq) {
@@ -298,8 +304,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         tc_commit(bar(L::kDsFree));
         if (next) {  // dP of the next Q tile once dQ_i has left the shared columns
-          if (kDq && !wait_bounded(bar(L::kDqFree), ph, limit_ns, abort_flag, err)) break;
-          if (!wait_bounded(bar(L::kDoFull + (it + 1) % DS), ((it + 1) / DS) & 1, limit_ns,
+          if (kDq && !wait_bounded_warp(bar(L::kDqFree), ph, limit_ns, abort_flag, err)) break;
+          if (!wait_bounded_warp(bar(L::kDoFull + (it + 1) % DS), ((it + 1) / DS) & 1, limit_ns,
                             abort_flag, err))
             break;
           tc_fence_after();
@@ -410,8 +416,10 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::kPReady));
 
-      // the previous tile's MMAs must be done reading dS^T
-      if (!wait_bounded_warp(bar(L::kDsFree), ph ^ 1, limit_ns, abort_flag, err) ||
+      // with dQ, dS^T goes to shared memory (dK and dQ read it there) once the
+      // previous tile's MMAs are done with it; without dQ it goes over the
+      // dP'^T columns just read, as bf16 pairs, and dK reads it from TMEM
+      if ((kDq && !wait_bounded_warp(bar(L::kDsFree), ph ^ 1, limit_ns, abort_flag, err)) ||
           !wait_bounded_warp(bar(L::kDpFull), ph, limit_ns, abort_flag, err)) {
         ok = false;
         break;
@@ -430,15 +438,22 @@ __global__ void __launch_bounds__(384, 1)
           w[e / 2] = pack_bf16x2(bf16_lo(pp) * __uint_as_float(u[e]),
                                  bf16_hi(pp) * __uint_as_float(u[e + 1]));
         }
+        if (kDq) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int qq = cc * 4 + q;  // 16-byte chunk index within the 256-byte row
-          st_shared_v4(dsrow + (qq >> 3) * 16384 + (((qq & 7) ^ (r & 7)) << 4), w[4 * q],
-                       w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          for (int q = 0; q < 4; ++q) {
+            const int qq = cc * 4 + q;  // 16-byte chunk index within the 256-byte row
+            st_shared_v4(dsrow + (qq >> 3) * 16384 + (((qq & 7) ^ (r & 7)) << 4), w[4 * q],
+                         w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          }
+        } else {
+          // packed columns h*64 + 16 cl .. +15, all already read (h = h0)
+          tmem_st_32x32b_x16(tmem + lane_off + L::kColDP + h0 * 64 + cl * 16,
+                             *reinterpret_cast<const uint32_t(*)[16]>(w));
         }
       }
+      if (!kDq) tmem_wait_st();
       tc_fence_before();
-      fence_proxy_async_smem();
+      if (kDq) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::kDsReady));
     }

@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // the whole warp runs this loop; the MMA and commit wrappers elect one lane
+    {
       constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t id_kmn = idesc_bf16_f32(128, D, false, true);
       const uint32_t err = err_k | kErrRoleMma;
@@ -170,9 +171,9 @@ __global__ void __launch_bounds__(384, 1)
         tc_commit(bar(L::kDpFull));
         tc_commit(bar(L::kVEmpty + (j % VS)));  // V_j is read only by dP_j
       };
-      bool ok = wait_bounded(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
-                wait_bounded(bar(L::kKFull), 0, limit_ns, abort_flag, err) &&
-                wait_bounded(bar(L::kVFull), 0, limit_ns, abort_flag, err);
+      bool ok = wait_bounded_warp(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
+                wait_bounded_warp(bar(L::kKFull), 0, limit_ns, abort_flag, err) &&
+                wait_bounded_warp(bar(L::kVFull), 0, limit_ns, abort_flag, err);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -182,13 +183,13 @@ __global__ void __launch_bounds__(384, 1)
         const int s = j % KS;
         const bool next = j + 1 < n_kv;
         if (next) {  // S_{j+1} into the region dQ_{j-1} has finished reading
-          if (!wait_bounded(bar(L::kKFull + (j + 1) % KS), ((j + 1) / KS) & 1, limit_ns,
+          if (!wait_bounded_warp(bar(L::kKFull + (j + 1) % KS), ((j + 1) / KS) & 1, limit_ns,
                             abort_flag, err))
             break;
           tc_fence_after();
           issue_s(j + 1);
         }
-        if (!wait_bounded(bar(L::kDsReady), j & 1, limit_ns, abort_flag, err)) break;
+        if (!wait_bounded_warp(bar(L::kDsReady), j & 1, limit_ns, abort_flag, err)) break;
         tc_fence_after();
         // dQ_i += dS_j K_j: A = dS_j from TMEM (keys 0-63 at columns 0-31 of
         // the region, keys 64-127 at columns 64-95), B = K_j MN-major
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(384, 1)
                       (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(L::kKEmpty + s));  // K_j: read by S_j and this dQ step
         if (next) {  // dP_{j+1}: the compute warps have read dP_j
-          if (!wait_bounded(bar(L::kVFull + (j + 1) % VS), ((j + 1) / VS) & 1, limit_ns,
+          if (!wait_bounded_warp(bar(L::kVFull + (j + 1) % VS), ((j + 1) / VS) & 1, limit_ns,
                             abort_flag, err))
             break;
           tc_fence_after();

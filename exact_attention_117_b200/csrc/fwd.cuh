@@ -195,7 +195,8 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
+      // the whole warp runs this loop; the MMA and commit wrappers elect one lane
+      {
         constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t id_o = idesc_bf16_f32(128, D, false, true);
         const uint32_t err = err_fwd | kErrRoleMma;
@@ -220,8 +221,8 @@ __global__ void __launch_bounds__(384, 1)
             mma_bf16_ts(d_tmem, a_tmem + kk * 8, sw128_desc(va + kk * 2048, 16384, 1024), id_o,
                         (jj > 0 || kk > 0) ? 1u : 0u);
         };
-        bool ok = n1 > 0 && wait_bounded(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
-                  wait_bounded(bar(L::kKFull), 0, limit_ns, abort_flag, err);
+        bool ok = n1 > 0 && wait_bounded_warp(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
+                  wait_bounded_warp(bar(L::kKFull), 0, limit_ns, abort_flag, err);
         if (ok) {
           tc_fence_after();
           if (n0 > 0) issue_s(0, 0);
@@ -230,9 +231,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int jj = 0; ok && jj < n1; ++jj) {
           const int s = jj % S;
-          if (!wait_bounded(bar(L::kVFull + s), (jj / S) & 1, limit_ns, abort_flag, err)) break;
+          if (!wait_bounded_warp(bar(L::kVFull + s), (jj / S) & 1, limit_ns, abort_flag, err)) break;
           if (jj < n0) {
-            if (!wait_bounded(bar(L::kPFull + 0), jj & 1, limit_ns, abort_flag, err)) break;
+            if (!wait_bounded_warp(bar(L::kPFull + 0), jj & 1, limit_ns, abort_flag, err)) break;
             tc_fence_after();
             issue_pv(0, jj);
             if (jj == n0 - 1) tc_commit(bar(L::kOFinal + 0));
@@ -240,12 +241,12 @@ __global__ void __launch_bounds__(384, 1)
           const bool next = jj + 1 < n1;
           const int s1 = (jj + 1) % S;
           if (next) {
-            if (!wait_bounded(bar(L::kKFull + s1), ((jj + 1) / S) & 1, limit_ns, abort_flag, err))
+            if (!wait_bounded_warp(bar(L::kKFull + s1), ((jj + 1) / S) & 1, limit_ns, abort_flag, err))
               break;
             tc_fence_after();
             if (jj + 1 < n0) issue_s(0, jj + 1);
           }
-          if (!wait_bounded(bar(L::kPFull + 1), jj & 1, limit_ns, abort_flag, err)) break;
+          if (!wait_bounded_warp(bar(L::kPFull + 1), jj & 1, limit_ns, abort_flag, err)) break;
           tc_fence_after();
           issue_pv(1, jj);
           if (jj == n1 - 1) tc_commit(bar(L::kOFinal + 1));
