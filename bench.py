@@ -3,6 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload c3|c4]
+    python bench.py --sweep all|c5|splitkv      (supplementary per-case lines)
+    python bench.py --traffic                   (cases for an ncu DRAM-bytes capture)
+    python bench.py --traffic-report NCU_CSV    (that capture against the traffic model)
 
 One step = the forward kernel (O, LSE) plus the backward (preprocess, main,
 dQ convert) on one batch of seeded synthetic bf16 inputs that are already
@@ -479,6 +482,87 @@ def run_sweep(args):
     fa.check_device_error(stream)
 
 
+TRAFFIC_N = (128, 256, 512, 1024, 2048, 4096)
+TRAFFIC_BH = 16  # B=1, H=16, d=128, full (non-causal) attention
+
+
+def run_traffic(args):
+    """One launch per case, for an ncu DRAM-bytes capture: for each N, the
+    forward kernel, then a naive attention that materialises S and P in HBM
+    (torch: S = (scale Q) K^T, P = softmax(S), O = P V, all bf16, three
+    kernels).  All inputs are created and synchronised before the first case,
+    so the captured kernels after the first ``fwd_kernel`` are exactly the cases,
+    in order."""
+    import torch
+
+    from exact_attention_117_b200 import fa
+    from exact_attention_117_b200.workloads import Workload, make_inputs
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    d = 128
+    cases = []
+    for n in TRAFFIC_N:
+        w = Workload(f"traffic_N{n}", 1, TRAFFIC_BH, n, d, seed_base=700 + n)
+        x = make_inputs(w, dev, with_do=False)
+        x["qs"] = (x["q"].float() * w.scale).to(torch.bfloat16)
+        x["kt"] = x["k"].transpose(-1, -2)
+        x["o"] = torch.empty_like(x["q"])
+        x["lse"] = torch.empty((1, TRAFFIC_BH, n), dtype=torch.float32, device=dev)
+        cases.append((w, x))
+    torch.cuda.synchronize()
+    for w, x in cases:
+        fa.forward(x["q"], x["k"], x["v"], causal=False, scale=w.scale, out=x["o"], lse=x["lse"])
+        s = torch.matmul(x["qs"], x["kt"])
+        p = torch.softmax(s, dim=-1)
+        torch.matmul(p, x["v"])
+        del s, p
+    torch.cuda.synchronize()
+    fa.check_device_error()
+    print(json.dumps({"traffic_cases": [w.N for w, _ in cases], "B": 1, "H": TRAFFIC_BH,
+                      "d": d}))
+
+
+def traffic_report(csv_path):
+    """Markdown table: ncu dram__bytes of each case against the page-2 traffic
+    model (oracle/traffic_model.py) times the B*H heads."""
+    import csv
+
+    from oracle.traffic_model import memory_work
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}
+    kernels = {}
+    with open(csv_path, newline="") as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    for row in csv.DictReader(lines):
+        k = kernels.setdefault(int(row["ID"]), {"name": row["Kernel Name"]})
+        k[row["Metric Name"]] = float(row["Metric Value"].replace(",", "")) * \
+            scale.get(row["Metric Unit"], 1)
+    seq = [kernels[i] for i in sorted(kernels)]
+    first = next(i for i, k in enumerate(seq) if "fwd_kernel" in k["name"])
+    groups = []
+    for k in seq[first:]:
+        if "fwd_kernel" in k["name"]:
+            groups.append({"fwd": k, "naive": []})
+        else:
+            groups[-1]["naive"].append(k)
+    rd, wr = "dram__bytes_read.sum", "dram__bytes_write.sum"
+    out = ["| N | fwd read MB (model / ncu) | fwd write MB (model / ncu) | "
+           "naive read MB (model / ncu) | naive write MB (model / ncu) | naive kernels |",
+           "|---|---|---|---|---|---|"]
+    for n, g in zip(TRAFFIC_N, groups):
+        m = memory_work(n, 128, elem_bytes=2, lse_bytes=4)
+        bh = TRAFFIC_BH
+        nr = sum(k.get(rd, 0) for k in g["naive"])
+        nw = sum(k.get(wr, 0) for k in g["naive"])
+        out.append(f"| {n} | {m['flash_read_bytes'] * bh / 1e6:.2f} / {g['fwd'].get(rd, 0) / 1e6:.2f}"
+                   f" | {m['flash_write_bytes'] * bh / 1e6:.2f} / {g['fwd'].get(wr, 0) / 1e6:.2f}"
+                   f" | {m['naive_read_bytes'] * bh / 1e6:.2f} / {nr / 1e6:.2f}"
+                   f" | {m['naive_write_bytes'] * bh / 1e6:.2f} / {nw / 1e6:.2f}"
+                   f" | {len(g['naive'])} |")
+    text = "\n".join(out)
+    print(text)
+    return text
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -491,9 +575,19 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--sweep", choices=["all", "c5", "splitkv"], default=None,
                     help="supplementary per-case measurements instead of the headline line")
+    ap.add_argument("--traffic", action="store_true",
+                    help="one launch per traffic-model case (run under ncu for DRAM bytes)")
+    ap.add_argument("--traffic-report", metavar="NCU_CSV", default=None,
+                    help="compare an ncu --csv capture of --traffic with the traffic model")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.traffic:
+        run_traffic(args)
+        return
+    if args.traffic_report:
+        traffic_report(args.traffic_report)
         return
 
     from exact_attention_117_b200.workloads import WORKLOADS
