@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload c3|c4]
-    python bench.py --sweep all|c5|splitkv      (supplementary per-case lines)
+    python bench.py --sweep all|c5|splitkv|kv_outer  (supplementary per-case lines)
     python bench.py --traffic                   (cases for an ncu DRAM-bytes capture)
     python bench.py --traffic-report NCU_CSV    (that capture against the traffic model)
 
@@ -460,6 +460,32 @@ def run_sweep(args):
                 ms = _time_device(step, flush, stream)
                 emit(f"{tag} fwd+bwd", (fwd_f + bwd_f) / (ms * 1e-3) / 1e12, ms)
             del x, o, lse, g, ws
+    if args.sweep in ("all", "kv_outer"):
+        # loop-order ablation: the forward with the Q tiles outside (fa_fwd)
+        # against the FlashAttention-1 order (KV tiles outside, one CTA per head)
+        for B, H, N, causal in ((2, 16, 4096, True), (2, 16, 4096, False), (8, 32, 1024, True)):
+            w = Workload(f"kv_outer_B{B}_H{H}_N{N}", B, H, N, 128, seed_base=600)
+            x = make_inputs(w, dev, with_do=False)
+            o = torch.empty_like(x["q"])
+            lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+            wsk = torch.empty(fa.kv_outer_workspace_size(B, H, N, 128), dtype=torch.uint8,
+                              device=dev)
+            fwd_f, _ = attention_flops(B, H, N, 128, causal)
+            tag = f"{w.name} d=128 {'causal' if causal else 'full'}"
+
+            def q_outer():
+                fa.forward(x["q"], x["k"], x["v"], causal=causal, out=o, lse=lse, stream=stream)
+
+            def kv_outer():
+                fa.forward_kv_outer(x["q"], x["k"], x["v"], causal=causal, out=o, lse=lse,
+                                    workspace=wsk, stream=stream)
+            for name, fn in (("fwd Q-outer", q_outer), ("fwd KV-outer", kv_outer)):
+                if args.once:
+                    fn()
+                    continue
+                ms = _time_device(fn, flush, stream)
+                emit(f"{tag} {name}", fwd_f / (ms * 1e-3) / 1e12, ms)
+            del x, o, lse, wsk
     if args.sweep in ("all", "splitkv"):
         for B, H, N, causal in ((1, 1, 16384, False), (1, 1, 16384, True), (1, 2, 32768, False),
                                 (1, 4, 8192, False)):
@@ -573,8 +599,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--sweep", choices=["all", "c5", "splitkv"], default=None,
+    ap.add_argument("--sweep", choices=["all", "c5", "splitkv", "kv_outer"], default=None,
                     help="supplementary per-case measurements instead of the headline line")
+    ap.add_argument("--once", action="store_true",
+                    help="with --sweep kv_outer: run each case once, untimed (for ncu)")
     ap.add_argument("--traffic", action="store_true",
                     help="one launch per traffic-model case (run under ncu for DRAM bytes)")
     ap.add_argument("--traffic-report", metavar="NCU_CSV", default=None,

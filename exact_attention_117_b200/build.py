@@ -13,7 +13,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfa_b200.so")
 SOURCES = ["fa_api.cu"]
-HEADERS = ["sm100.cuh", "common.cuh", "fwd.cuh", "bwd.cuh", "bwd_main.cuh", "dq_pass.cuh"]
+HEADERS = ["sm100.cuh", "common.cuh", "fwd.cuh", "bwd.cuh", "bwd_main.cuh", "dq_pass.cuh", "kv_outer.cuh"]
 
 
 def nvcc() -> str:

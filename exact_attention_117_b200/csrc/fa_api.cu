@@ -16,6 +16,7 @@
 #include "../../include/fa.h"
 #include "bwd.cuh"
 #include "fwd.cuh"
+#include "kv_outer.cuh"
 
 namespace {
 
@@ -260,6 +261,44 @@ fa_status bwd_entry(const void* q, const void* k, const void* v, const void* o, 
                                                ws, bh, N, scale, s);
 }
 
+struct KvOuterWorkspace {
+  float* o_acc;
+  float* m;
+  float* l;
+  size_t bytes;
+};
+
+KvOuterWorkspace kv_outer_layout(void* base, int B, int H, int N, int d) {
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t np = round_up(static_cast<size_t>(N), 128);
+  const size_t acc = round_up(bh * np * d * sizeof(float), 256);
+  const size_t vec = round_up(bh * np * sizeof(float), 256);
+  char* p = static_cast<char*>(base);
+  return {reinterpret_cast<float*>(p), reinterpret_cast<float*>(p + acc),
+          reinterpret_cast<float*>(p + acc + vec), acc + 2 * vec};
+}
+
+template <int D, bool C>
+fa_status launch_kv_outer(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const CUtensorMap& mo, float* lse, const KvOuterWorkspace& ws, int BH,
+                          int N, float scale_log2, cudaStream_t st) {
+  using L = fa::KvOuterLayout<D>;
+  static bool attr_set[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return FA_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (!set_smem(fa::kv_outer_fwd_kernel<D, C>, L::kSmemAlloc)) return FA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  const int np = static_cast<int>(round_up(static_cast<size_t>(N), 128));
+  {
+    LaunchTimer timer(st, FA_KERNEL_FWD_KV_OUTER);
+    fa::kv_outer_fwd_kernel<D, C><<<static_cast<unsigned>(BH), 256, L::kSmemAlloc, st>>>(
+        mq, mk, mv, mo, lse, ws.o_acc, ws.m, ws.l, N, np, scale_log2, kWaitLimitNs);
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -340,6 +379,37 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
           part_o, part_lse, static_cast<__nv_bfloat16*>(o), lse, bh, N, num_splits);
   }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_fwd_kv_outer_workspace_size(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.0f) != FA_OK) return 0;
+  return kv_outer_layout(nullptr, B, H, N, d).bytes;
+}
+
+fa_status fa_fwd_kv_outer(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int H, int N, int d, int causal, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  fa_status st = check_common(B, H, N, d, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGN;
+  const KvOuterWorkspace ws = kv_outer_layout(workspace, B, H, N, d);
+  if (!workspace || workspace_bytes < ws.bytes) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGN;
+  const int bh = B * H;
+  CUtensorMap mq, mk, mv, mo;
+  if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
+      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mo, o, d, N, bh, 128))
+    return FA_ERR_CUDA;
+  const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return causal ? launch_kv_outer<64, true>(mq, mk, mv, mo, lse, ws, bh, N, scale_log2, s)
+                  : launch_kv_outer<64, false>(mq, mk, mv, mo, lse, ws, bh, N, scale_log2, s);
+  return causal ? launch_kv_outer<128, true>(mq, mk, mv, mo, lse, ws, bh, N, scale_log2, s)
+                : launch_kv_outer<128, false>(mq, mk, mv, mo, lse, ws, bh, N, scale_log2, s);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

@@ -24,7 +24,7 @@ STATUS_NAMES = {
     4: "FA_ERR_ALIGN", 5: "FA_ERR_SCALE", 6: "FA_ERR_WORKSPACE", 7: "FA_ERR_CUDA",
     8: "FA_ERR_DEVICE_TIMEOUT", 9: "FA_ERR_STATE",
 }
-KERNELS = ("fwd", "bwd_pre", "bwd_main", "bwd_dq", "fwd_combine")
+KERNELS = ("fwd", "bwd_pre", "bwd_main", "bwd_dq", "fwd_combine", "fwd_kv_outer")
 
 _lib = None
 
@@ -52,6 +52,10 @@ def load() -> ctypes.CDLL:
     lib.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i]
     lib.fa_fwd_splitkv.restype = i
     lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_fwd_kv_outer_workspace_size.restype = sz
+    lib.fa_fwd_kv_outer_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_fwd_kv_outer.restype = i
+    lib.fa_fwd_kv_outer.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd.restype = i
@@ -164,6 +168,30 @@ def bwd_deterministic_raw(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, H, N
     """Direct call of ``fa_bwd_deterministic`` with raw pointers; returns the status code."""
     return load().fa_bwd_deterministic(q, k, v, o, lse, do, dq, dk, dv, ws, ws_bytes, B, H, N, d,
                                        int(bool(causal)), float(scale), stream)
+
+
+def kv_outer_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load().fa_fwd_kv_outer_workspace_size(B, H, N, d))
+
+
+def forward_kv_outer(q, k, v, causal: bool = False, scale: Optional[float] = None, out=None,
+                     lse=None, workspace=None, stream=None):
+    """O, LSE through the KV-outer (FlashAttention-1 order) forward kernel."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = kv_outer_workspace_size(B, H, N, d)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(load().fa_fwd_kv_outer(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
+                                  int(bool(causal)), float(scale), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(),
+                                  _stream_ptr(stream)), "fa_fwd_kv_outer")
+    return out, lse
 
 
 def backward(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None,

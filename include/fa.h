@@ -186,6 +186,37 @@ FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, con
                                 void* stream);
 
 /*
+ * Forward in the FlashAttention-1 loop order, for measurement (a loop-order
+ * ablation): same arguments, preconditions and results as fa_fwd, up to
+ * rounding, plus a workspace.
+ *
+ * Page "从零实现 FlashAttention-2：分块在线 Softmax", section 从 FlashAttention-1
+ * 到 FlashAttention-2: the first version loops over key/value tiles outside
+ * and query tiles inside; the second swaps the loops (fa_fwd) and also
+ * parallelises over the sequence.  Here one CTA per (batch, head) loads each
+ * K/V tile once and, for every query tile that sees it, reads Q_i and the
+ * running row statistics m_i, l_i and output O_i (fp32, in the workspace) from
+ * global memory, merges the tile's contribution with the page-3 rule
+ * ("FlashAttention 为什么能节省显存并提速,是否改变注意力结果?", section
+ * 难点在于分块后softmax如何归一) and writes them back; bf16 O and LSE are
+ * written after the last key tile.  It is slower than fa_fwd by design: the
+ * extra reads and writes of O_i per (i, j) step and the B*H-CTA grid are what
+ * it measures.
+ *
+ *   workspace : device scratch of at least fa_fwd_kv_outer_workspace_size
+ *               bytes (fp32 O of B*H*Np*d floats, then m and l of B*H*Np
+ *               floats each, Np = N rounded up to 128), 16-byte aligned; its
+ *               contents on entry do not matter.
+ * Returns the same codes as fa_fwd, and FA_ERR_WORKSPACE for a missing or
+ * short workspace.
+ */
+FA_API size_t fa_fwd_kv_outer_workspace_size(int B, int H, int N, int d);
+FA_API fa_status fa_fwd_kv_outer(const void* q, const void* k, const void* v, void* o,
+                                 float* lse, int B, int H, int N, int d, int causal,
+                                 float scale, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  Returns FA_OK, FA_ERR_DEVICE_TIMEOUT (a bounded wait ran
  * out; *detail, if non-NULL, receives which one) or FA_ERR_CUDA.
@@ -212,9 +243,11 @@ typedef enum {
   FA_KERNEL_FWD = 0,       /* forward kernel                         */
   FA_KERNEL_BWD_PRE = 1,   /* backward: D = rowsum(dO*O), clears dQ  */
   FA_KERNEL_BWD_MAIN = 2,  /* backward: per-KV-tile main kernel      */
-  FA_KERNEL_BWD_DQ = 3,    /* backward: dQ fp32 -> bf16              */
+  FA_KERNEL_BWD_DQ = 3,    /* backward: dQ fp32 -> bf16 (fa_bwd), or the
+                              dQ pass (fa_bwd_deterministic)         */
   FA_KERNEL_FWD_COMBINE = 4, /* split-KV forward: merge of the splits */
-  FA_KERNEL_COUNT = 5
+  FA_KERNEL_FWD_KV_OUTER = 5, /* forward in the KV-outer loop order    */
+  FA_KERNEL_COUNT = 6
 } fa_kernel_id;
 
 /*
