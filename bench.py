@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload c3|c4]
-    python bench.py --sweep all|c5|splitkv|kv_outer  (supplementary per-case lines)
+    python bench.py --sweep all|c5|splitkv|kv_outer|bwd  (supplementary per-case lines)
     python bench.py --traffic                   (cases for an ncu DRAM-bytes capture)
     python bench.py --traffic-report NCU_CSV    (that capture against the traffic model)
 
@@ -460,6 +460,41 @@ def run_sweep(args):
                 ms = _time_device(step, flush, stream)
                 emit(f"{tag} fwd+bwd", (fwd_f + bwd_f) / (ms * 1e-3) / 1e12, ms)
             del x, o, lse, g, ws
+    if args.sweep in ("all", "bwd"):
+        # the two backward variants on the headline workloads: fa_bwd (dQ by
+        # fp32 atomics) and fa_bwd_deterministic (dQ by a query-tile pass)
+        from exact_attention_117_b200.workloads import WORKLOADS
+        for name in (("c3",) if args.once else ("c3", "c4")):
+            w = WORKLOADS[name]
+            x = make_inputs(w, dev)
+            o = torch.empty_like(x["q"])
+            lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+            g = [torch.empty_like(x["q"]) for _ in range(3)]
+            ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+            fwd_f, bwd_f = attention_flops(w.B, w.H, w.N, w.d, True)
+
+            def fwd():
+                fa.forward(x["q"], x["k"], x["v"], causal=True, out=o, lse=lse, stream=stream)
+
+            def bwd(det):
+                fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=True, dq=g[0],
+                            dk=g[1], dv=g[2], workspace=ws, stream=stream, deterministic=det)
+            if args.once:  # two rounds of fwd, atomic bwd, deterministic bwd (for ncu)
+                for _ in range(2):
+                    fwd()
+                    bwd(False)
+                    bwd(True)
+                continue
+            ms = _time_device(fwd, flush, stream)
+            emit(f"{name} causal fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
+            for det in (False, True):
+                fwd()
+                with fa.KernelTimer() as kt:
+                    ms = _time_device(lambda: bwd(det), flush, stream)
+                per = {k: round(kt.ms[k] / kt.launches[k], 4) for k in kt.ms if kt.launches[k]}
+                emit(f"{name} causal bwd {'deterministic' if det else 'atomic dQ'} "
+                     f"(per-kernel ms {per})", bwd_f / (ms * 1e-3) / 1e12, ms)
+            del x, o, lse, g, ws
     if args.sweep in ("all", "kv_outer"):
         # loop-order ablation: the forward with the Q tiles outside (fa_fwd)
         # against the FlashAttention-1 order (KV tiles outside, one CTA per head)
@@ -599,10 +634,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--sweep", choices=["all", "c5", "splitkv", "kv_outer"], default=None,
+    ap.add_argument("--sweep", choices=["all", "c5", "splitkv", "kv_outer", "bwd"], default=None,
                     help="supplementary per-case measurements instead of the headline line")
     ap.add_argument("--once", action="store_true",
-                    help="with --sweep kv_outer: run each case once, untimed (for ncu)")
+                    help="with --sweep kv_outer or bwd: run the cases once, untimed (for ncu)")
     ap.add_argument("--traffic", action="store_true",
                     help="one launch per traffic-model case (run under ncu for DRAM bytes)")
     ap.add_argument("--traffic-report", metavar="NCU_CSV", default=None,
