@@ -206,6 +206,14 @@ def oracle_sample(w, budget_s, device_inputs=None):
                     f"({t_total:.1f} s)")
 
 
+def line_config(w):
+    """The ``config`` object of the JSON line; both arms print the same one."""
+    return {"workload": f"{w.name}: causal fwd+bwd, B={w.B} H={w.H} N={w.N} d={w.d}",
+            "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "scale": w.scale,
+            "per_rank": "independent copy of the batch on every rank",
+            "l2": "flushed (256 MiB write) before every timed step, outside its events"}
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return
@@ -228,8 +236,7 @@ def run_reference(args, w, rank):
         "n_gpus": args.gpus, "steps": steps, "warmup": warm,
         "ms_per_step": 1000.0 * wall / steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True,
-                   "sample": "bounded per-step sample of (b,h) slices"},
+        "config": line_config(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
                          "kind": "oracle", "sample": descs[-1]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -381,10 +388,7 @@ def run_ours(args, w, rank, world, local_rank):
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: causal fwd+bwd, B={B} H={H} N={N} d={d}",
-                   "B": B, "H": H, "N": N, "d": d, "causal": True, "scale": w.scale,
-                   "per_rank": "independent copy of the batch on every rank",
-                   "l2": "flushed (256 MiB write) before every timed step, outside its events"},
+        "config": line_config(w),
         "fwd": {"ms": fwd_ms_per, "tflops": fwd_f / (fwd_ms_per * 1e-3) / 1e12,
                 "kernel_tflops": fwd_tf, "pct_of_peak": 100.0 * (fwd_tf or 0) / peak_tf},
         "bwd": {"ms": bwd_ms_per, "tflops": bwd_tf, "pct_of_peak": 100.0 * bwd_tf / peak_tf},
