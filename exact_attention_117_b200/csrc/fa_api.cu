@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -123,6 +124,19 @@ bool set_smem(K kernel, int bytes) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Number of SMs of device `dev` (looked up once per device).
+int sm_count(int dev) {
+  static int count[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (count[dev] == 0) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
+      c = 148;
+    count[dev] = c;
+  }
+  return count[dev];
+}
+
 struct BwdWorkspace {
   float* dq_acc;  // [BH, Np, d]
   float* dvec;    // [BH, Np]
@@ -195,7 +209,11 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   {
     LaunchTimer timer(st, FA_KERNEL_BWD_PRE);
     const long long rows = static_cast<long long>(BH) * np;
-    const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);  // 8 rows (warps) per block
+    const long long rows_per_warp = 4LL * (32 / (D / 8));  // see bwd_preprocess_kernel
+    const long long warps = (rows + rows_per_warp - 1) / rows_per_warp;
+    // a grid-stride kernel: at most 8 blocks of 8 warps per SM
+    const long long cap = 8LL * sm_count(dev);
+    const unsigned blocks = static_cast<unsigned>(std::min((warps + 7) / 8, cap));
     fa::bwd_preprocess_kernel<D><<<blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
         ws.dvec, ws.lse2, kDet ? nullptr : ws.dq_acc, BH, N, np,
@@ -217,8 +235,8 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
         mq, mk, mv, mdo, mdq, ws.dvec, ws.lse2, N, np, scale, scale_log2, kWaitLimitNs);
   } else {
     LaunchTimer timer(st, FA_KERNEL_BWD_DQ);
-    const long long elems = static_cast<long long>(BH) * N * D;
-    const unsigned blocks = static_cast<unsigned>((elems / 8 + 255) / 256);
+    const long long warps = (static_cast<long long>(BH) * N + 15) / 16 * (D / 16);
+    const unsigned blocks = static_cast<unsigned>((warps + 7) / 8);  // 8 warps per block
     fa::dq_convert_kernel<D><<<blocks, 256, 0, st>>>(ws.dq_acc, static_cast<__nv_bfloat16*>(dq),
                                                       BH, N, np, scale);
   }
