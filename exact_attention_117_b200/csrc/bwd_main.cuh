@@ -21,10 +21,12 @@
 // does the per-column subtraction and the softmax threads load no per-column
 // values.  Warp 2 builds those slabs from LSE2 and D in global memory.
 //
-// Issue order of the tensor-core work: ... dV_i, S_{i+1}, dK_i, dQ_i, dP_{i+1},
+// Issue order of the tensor-core work: ... dV_i, S_{i+1}, dQ_i, dK_i, dP_{i+1},
 // dV_{i+1} ...  S_{i+1} goes right after dV_i (tcgen05.mma ops of one thread
 // run in order, so it cannot overwrite P_i before dV_i has read it), which lets
-// the exponentials of tile i+1 overlap dK_i and dQ_i on the tensor core.
+// the exponentials of tile i+1 overlap dQ_i and dK_i on the tensor core; dQ_i
+// goes before dK_i so that its read-out overlaps dK_i and dP_{i+1}, which
+// reuses its TMEM columns, is not held up.
 //
 // dK_j and dV_j accumulate in TMEM and are written once by this CTA (no
 // atomics), staged through shared memory and stored with TMA; dQ_i partial
@@ -282,6 +284,15 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!wait_bounded_warp(bar(L::kDsReady), ph, limit_ns, abort_flag, err)) break;
         tc_fence_after();
+        // dQ_i first: its read-out (and the dP_{i+1} that reuses its columns)
+        // then overlaps dK_i
+        if (kDq) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // dQ_i = dS K_j  (K = 128 keys)
+            mma_bf16_ss(tmem + L::kColDQ, sw128_desc(a_ds + kk * 2048, 16384, 1024),
+                        sw128_desc(a_k + kk * 2048, 16384, 1024), id_mnmn, kk > 0 ? 1u : 0u);
+          tc_commit(bar(L::kDqFull));
+        }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {  // dK_j += dS^T Q_i
           const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
@@ -295,13 +306,6 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         tc_commit(bar(L::kQEmpty + st));  // Q_i and its slab are no longer read
-        if (kDq) {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // dQ_i = dS K_j  (K = 128 keys)
-            mma_bf16_ss(tmem + L::kColDQ, sw128_desc(a_ds + kk * 2048, 16384, 1024),
-                        sw128_desc(a_k + kk * 2048, 16384, 1024), id_mnmn, kk > 0 ? 1u : 0u);
-          tc_commit(bar(L::kDqFull));
-        }
         tc_commit(bar(L::kDsFree));
         if (next) {  // dP of the next Q tile once dQ_i has left the shared columns
           if (kDq && !wait_bounded_warp(bar(L::kDqFree), ph, limit_ns, abort_flag, err)) break;
