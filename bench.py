@@ -441,109 +441,134 @@ def run_sweep(args):
         print(json.dumps({"sweep": case, "tflops": round(tflops, 1), "ms": round(ms, 4),
                           "pct_of_peak": round(100 * tflops / peak, 1)}), flush=True)
 
+    class category:
+        """Samples the SM clocks while one group of cases runs and prints them
+        (a throttled group shows as a low median or an active reason)."""
+
+        def __init__(self, name):
+            self.name = name
+            self.clk = ClockSampler(0)
+
+        def __enter__(self):
+            self.clk.__enter__()
+            return self
+
+        def __exit__(self, *exc):
+            self.clk.__exit__(*exc)
+            if not args.once:
+                print(json.dumps({"sweep_clocks": self.name, **self.clk.summary()}), flush=True)
+            return False
+
     if args.sweep in ("all", "c5"):
-        for w in sweep_workloads():
-            x = make_inputs(w, dev)
-            o = torch.empty_like(x["q"])
-            lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
-            g = [torch.empty_like(x["q"]) for _ in range(3)]
-            ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
-            for causal in (True, False):
-                fwd_f, bwd_f = attention_flops(w.B, w.H, w.N, w.d, causal)
+        with category("c5"):
+            for w in sweep_workloads():
+                x = make_inputs(w, dev)
+                o = torch.empty_like(x["q"])
+                lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+                g = [torch.empty_like(x["q"]) for _ in range(3)]
+                ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8,
+                                 device=dev)
+                for causal in (True, False):
+                    fwd_f, bwd_f = attention_flops(w.B, w.H, w.N, w.d, causal)
+
+                    def fwd():
+                        fa.forward(x["q"], x["k"], x["v"], causal=causal, out=o, lse=lse,
+                                   stream=stream)
+
+                    def step():
+                        fwd()
+                        fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal,
+                                    dq=g[0], dk=g[1], dv=g[2], workspace=ws, stream=stream)
+                    tag = f"{w.name} {'causal' if causal else 'full'}"
+                    ms = _time_device(fwd, flush, stream)
+                    emit(f"{tag} fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
+                    ms = _time_device(step, flush, stream)
+                    emit(f"{tag} fwd+bwd", (fwd_f + bwd_f) / (ms * 1e-3) / 1e12, ms)
+                del x, o, lse, g, ws
+    if args.sweep in ("all", "bwd"):
+        with category("bwd"):
+            # the two backward variants on the headline workloads: fa_bwd (dQ by
+            # fp32 atomics) and fa_bwd_deterministic (dQ by a query-tile pass)
+            from exact_attention_117_b200.workloads import WORKLOADS
+            for name in (("c3",) if args.once else ("c3", "c4")):
+                w = WORKLOADS[name]
+                x = make_inputs(w, dev)
+                o = torch.empty_like(x["q"])
+                lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+                g = [torch.empty_like(x["q"]) for _ in range(3)]
+                ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8,
+                                 device=dev)
+                fwd_f, bwd_f = attention_flops(w.B, w.H, w.N, w.d, True)
 
                 def fwd():
+                    fa.forward(x["q"], x["k"], x["v"], causal=True, out=o, lse=lse, stream=stream)
+
+                def bwd(det):
+                    fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=True, dq=g[0],
+                                dk=g[1], dv=g[2], workspace=ws, stream=stream, deterministic=det)
+                if args.once:  # two rounds of fwd, atomic bwd, deterministic bwd (for ncu)
+                    for _ in range(2):
+                        fwd()
+                        bwd(False)
+                        bwd(True)
+                    continue
+                ms = _time_device(fwd, flush, stream)
+                emit(f"{name} causal fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
+                for det in (False, True):
+                    fwd()
+                    with fa.KernelTimer() as kt:
+                        ms = _time_device(lambda: bwd(det), flush, stream)
+                    per = {k: round(kt.ms[k] / kt.launches[k], 4) for k in kt.ms if kt.launches[k]}
+                    emit(f"{name} causal bwd {'deterministic' if det else 'atomic dQ'} "
+                         f"(per-kernel ms {per})", bwd_f / (ms * 1e-3) / 1e12, ms)
+                del x, o, lse, g, ws
+    if args.sweep in ("all", "kv_outer"):
+        with category("kv_outer"):
+            # loop-order ablation: the forward with the Q tiles outside (fa_fwd)
+            # against the FlashAttention-1 order (KV tiles outside, one CTA per head)
+            for B, H, N, causal in ((2, 16, 4096, True), (2, 16, 4096, False), (8, 32, 1024, True)):
+                w = Workload(f"kv_outer_B{B}_H{H}_N{N}", B, H, N, 128, seed_base=600)
+                x = make_inputs(w, dev, with_do=False)
+                o = torch.empty_like(x["q"])
+                lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+                wsk = torch.empty(fa.kv_outer_workspace_size(B, H, N, 128), dtype=torch.uint8,
+                                  device=dev)
+                fwd_f, _ = attention_flops(B, H, N, 128, causal)
+                tag = f"{w.name} d=128 {'causal' if causal else 'full'}"
+
+                def q_outer():
                     fa.forward(x["q"], x["k"], x["v"], causal=causal, out=o, lse=lse, stream=stream)
 
-                def step():
-                    fwd()
-                    fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal,
-                                dq=g[0], dk=g[1], dv=g[2], workspace=ws, stream=stream)
-                tag = f"{w.name} {'causal' if causal else 'full'}"
-                ms = _time_device(fwd, flush, stream)
-                emit(f"{tag} fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
-                ms = _time_device(step, flush, stream)
-                emit(f"{tag} fwd+bwd", (fwd_f + bwd_f) / (ms * 1e-3) / 1e12, ms)
-            del x, o, lse, g, ws
-    if args.sweep in ("all", "bwd"):
-        # the two backward variants on the headline workloads: fa_bwd (dQ by
-        # fp32 atomics) and fa_bwd_deterministic (dQ by a query-tile pass)
-        from exact_attention_117_b200.workloads import WORKLOADS
-        for name in (("c3",) if args.once else ("c3", "c4")):
-            w = WORKLOADS[name]
-            x = make_inputs(w, dev)
-            o = torch.empty_like(x["q"])
-            lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
-            g = [torch.empty_like(x["q"]) for _ in range(3)]
-            ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
-            fwd_f, bwd_f = attention_flops(w.B, w.H, w.N, w.d, True)
-
-            def fwd():
-                fa.forward(x["q"], x["k"], x["v"], causal=True, out=o, lse=lse, stream=stream)
-
-            def bwd(det):
-                fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=True, dq=g[0],
-                            dk=g[1], dv=g[2], workspace=ws, stream=stream, deterministic=det)
-            if args.once:  # two rounds of fwd, atomic bwd, deterministic bwd (for ncu)
-                for _ in range(2):
-                    fwd()
-                    bwd(False)
-                    bwd(True)
-                continue
-            ms = _time_device(fwd, flush, stream)
-            emit(f"{name} causal fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
-            for det in (False, True):
-                fwd()
-                with fa.KernelTimer() as kt:
-                    ms = _time_device(lambda: bwd(det), flush, stream)
-                per = {k: round(kt.ms[k] / kt.launches[k], 4) for k in kt.ms if kt.launches[k]}
-                emit(f"{name} causal bwd {'deterministic' if det else 'atomic dQ'} "
-                     f"(per-kernel ms {per})", bwd_f / (ms * 1e-3) / 1e12, ms)
-            del x, o, lse, g, ws
-    if args.sweep in ("all", "kv_outer"):
-        # loop-order ablation: the forward with the Q tiles outside (fa_fwd)
-        # against the FlashAttention-1 order (KV tiles outside, one CTA per head)
-        for B, H, N, causal in ((2, 16, 4096, True), (2, 16, 4096, False), (8, 32, 1024, True)):
-            w = Workload(f"kv_outer_B{B}_H{H}_N{N}", B, H, N, 128, seed_base=600)
-            x = make_inputs(w, dev, with_do=False)
-            o = torch.empty_like(x["q"])
-            lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-            wsk = torch.empty(fa.kv_outer_workspace_size(B, H, N, 128), dtype=torch.uint8,
-                              device=dev)
-            fwd_f, _ = attention_flops(B, H, N, 128, causal)
-            tag = f"{w.name} d=128 {'causal' if causal else 'full'}"
-
-            def q_outer():
-                fa.forward(x["q"], x["k"], x["v"], causal=causal, out=o, lse=lse, stream=stream)
-
-            def kv_outer():
-                fa.forward_kv_outer(x["q"], x["k"], x["v"], causal=causal, out=o, lse=lse,
-                                    workspace=wsk, stream=stream)
-            for name, fn in (("fwd Q-outer", q_outer), ("fwd KV-outer", kv_outer)):
-                if args.once:
-                    fn()
-                    continue
-                ms = _time_device(fn, flush, stream)
-                emit(f"{tag} {name}", fwd_f / (ms * 1e-3) / 1e12, ms)
-            del x, o, lse, wsk
+                def kv_outer():
+                    fa.forward_kv_outer(x["q"], x["k"], x["v"], causal=causal, out=o, lse=lse,
+                                        workspace=wsk, stream=stream)
+                for name, fn in (("fwd Q-outer", q_outer), ("fwd KV-outer", kv_outer)):
+                    if args.once:
+                        fn()
+                        continue
+                    ms = _time_device(fn, flush, stream)
+                    emit(f"{tag} {name}", fwd_f / (ms * 1e-3) / 1e12, ms)
+                del x, o, lse, wsk
     if args.sweep in ("all", "splitkv"):
-        for B, H, N, causal in ((1, 1, 16384, False), (1, 1, 16384, True), (1, 2, 32768, False),
-                                (1, 4, 8192, False)):
-            w = Workload(f"few_heads_B{B}_H{H}_N{N}", B, H, N, 128, seed_base=500)
-            x = make_inputs(w, dev, with_do=False)
-            o = torch.empty_like(x["q"])
-            lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-            fwd_f, _ = attention_flops(B, H, N, 128, causal)
-            tag = f"{w.name} d=128 {'causal' if causal else 'full'}"
-            ms = _time_device(lambda: fa.forward(x["q"], x["k"], x["v"], causal=causal, out=o,
-                                                 lse=lse, stream=stream), flush, stream)
-            emit(f"{tag} fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
-            for splits in (2, 4, 8):
-                wsz = fa.splitkv_workspace_size(B, H, N, 128, splits)
-                wsp = torch.empty(wsz, dtype=torch.uint8, device=dev)
-                ms = _time_device(lambda: fa.forward_splitkv(
-                    x["q"], x["k"], x["v"], causal=causal, num_splits=splits, out=o, lse=lse,
-                    workspace=wsp, stream=stream), flush, stream)
-                emit(f"{tag} fwd split-KV x{splits}", fwd_f / (ms * 1e-3) / 1e12, ms)
+        with category("splitkv"):
+            for B, H, N, causal in ((1, 1, 16384, False), (1, 1, 16384, True), (1, 2, 32768, False),
+                                    (1, 4, 8192, False)):
+                w = Workload(f"few_heads_B{B}_H{H}_N{N}", B, H, N, 128, seed_base=500)
+                x = make_inputs(w, dev, with_do=False)
+                o = torch.empty_like(x["q"])
+                lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+                fwd_f, _ = attention_flops(B, H, N, 128, causal)
+                tag = f"{w.name} d=128 {'causal' if causal else 'full'}"
+                ms = _time_device(lambda: fa.forward(x["q"], x["k"], x["v"], causal=causal, out=o,
+                                                     lse=lse, stream=stream), flush, stream)
+                emit(f"{tag} fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
+                for splits in (2, 4, 8):
+                    wsz = fa.splitkv_workspace_size(B, H, N, 128, splits)
+                    wsp = torch.empty(wsz, dtype=torch.uint8, device=dev)
+                    ms = _time_device(lambda: fa.forward_splitkv(
+                        x["q"], x["k"], x["v"], causal=causal, num_splits=splits, out=o, lse=lse,
+                        workspace=wsp, stream=stream), flush, stream)
+                    emit(f"{tag} fwd split-KV x{splits}", fwd_f / (ms * 1e-3) / 1e12, ms)
     fa.check_device_error(stream)
 
 
