@@ -88,14 +88,23 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _strip_comments(text):
+    """C++ source without comments and trailing blanks (what the compiler sees)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
 def source_digest():
-    """Hash of the kernel sources: ncu counters are only valid for this exact code."""
+    """Hash of the kernel code (comments excluded): ncu counters are only valid
+    for this exact code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_attention_117_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

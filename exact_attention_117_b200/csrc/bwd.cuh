@@ -16,6 +16,9 @@
 //                           it; dQ_i partial sums go to the fp32 accumulator
 //                           with vector atomic adds
 //   dq_convert_kernel     : dQ = bf16(scale * accumulator)
+// The deterministic backward runs bwd_main_kernel without its dQ part, then
+// dq_pass_kernel (dq_pass.cuh) in place of dq_convert_kernel: one CTA per
+// 128-row Q tile sums dQ over the key tiles in a fixed order and writes it.
 #pragma once
 
 #include <cuda_bf16.h>

@@ -150,3 +150,15 @@ def test_bench_traffic_report_parses_ncu_csv(tmp_path):
     lines = text.splitlines()
     assert len(lines) == 2 + len(bench.TRAFFIC_N)
     assert lines[2].startswith("| 128 |") and "/ 2.00" in lines[2] and "/ 30.00" in lines[2]
+
+
+def test_source_digest_ignores_comments_only():
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    a = "int a = 1;  // one\n/* block\n comment */\nint b = a;\n"
+    b = "// header\nint a = 1;\n\nint b = a;   \n"
+    c = "int a = 2;\nint b = a;\n"
+    assert bench._strip_comments(a) == bench._strip_comments(b)
+    assert bench._strip_comments(a) != bench._strip_comments(c)
