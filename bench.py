@@ -123,30 +123,64 @@ def ncu_traffic(kernel_key, workload):
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+    """Samples the SM clock and the clock-event (throttle) reasons while the
+    timed region runs: through NVML (read-only queries) from a thread, first as
+    the region starts and then every 20 ms, or through nvidia-smi every 200 ms
+    where NVML is missing.  Sampling is kept sparse on purpose: NVML queries
+    issued once per step from the launching thread slowed the timed kernels
+    by 4 % on B200 (measured A/B)."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("sw_power_cap", "hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown")
+    BITS = (0x4, 0x8, 0x20, 0x40)  # nvmlClocksEventReason{SwPowerCap,HwSlowdown,Sw/HwThermal}
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
-        self.samples = []
+        self.samples = []  # (sm_mhz, max_mhz, set of active reasons)
+        self.source = None
         self._stop = threading.Event()
         self._t = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._handle = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self._nvml = pynvml
+            self.source = "nvml"
+        except Exception:
+            self.source = "nvidia-smi"
+
+    def _sample_nvml(self):
+        nv, h = self._nvml, self._handle
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        bits = get(h)
+        self.samples.append((float(sm), float(mx),
+                             {n for n, b in zip(self.NAMES, self.BITS) if bits & b}))
+
+    def _sample_smi(self):
+        out = subprocess.run(
+            ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.SMI_FIELDS}",
+             "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+        p = [x.strip() for x in out.stdout.strip().split(",")]
+        if len(p) == 7 and p[0].replace(".", "").isdigit() and p[1].replace(".", "").isdigit():
+            act = {"hw_slowdown": p[3], "hw_thermal_slowdown": p[4],
+                   "sw_thermal_slowdown": p[5], "sw_power_cap": p[6]}
+            self.samples.append((float(p[0]), float(p[1]),
+                                 {k for k, v in act.items() if v.lower() == "active"}))
 
     def _run(self):
+        period = 0.02 if self._nvml else 0.2
         while not self._stop.is_set():
             try:
-                out = subprocess.run(
-                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                     "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-                parts = [x.strip() for x in out.stdout.strip().split(",")]
-                if len(parts) == 7:
-                    self.samples.append(parts)
+                self._sample_nvml() if self._nvml else self._sample_smi()
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            self._stop.wait(period)
 
     def __enter__(self):
         self._t = threading.Thread(target=self._run, daemon=True)
@@ -160,15 +194,12 @@ class ClockSampler:
 
     def summary(self):
         if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if s[3 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"],
+                    "source": self.source}
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples),
+                "reasons": sorted(set().union(*(s[2] for s in self.samples))),
+                "samples": len(self.samples), "source": self.source}
 
 
 def cpu_threads():

@@ -162,3 +162,33 @@ def test_source_digest_ignores_comments_only():
     c = "int a = 2;\nint b = a;\n"
     assert bench._strip_comments(a) == bench._strip_comments(b)
     assert bench._strip_comments(a) != bench._strip_comments(c)
+
+
+def test_clock_sampler_decodes_nvml_reasons():
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+
+    class FakeNvml:  # read-only queries of a GPU at 1800 of 1965 MHz under the power cap
+        NVML_CLOCK_SM = 1
+
+        @staticmethod
+        def nvmlDeviceGetClockInfo(h, kind):
+            return 1800
+
+        @staticmethod
+        def nvmlDeviceGetMaxClockInfo(h, kind):
+            return 1965
+
+        @staticmethod
+        def nvmlDeviceGetCurrentClocksEventReasons(h):
+            return 0x4 | 0x1  # sw power cap, plus the (ignored) idle bit
+
+    c = bench.ClockSampler(0)
+    c._nvml, c._handle, c.source = FakeNvml, object(), "nvml"
+    for _ in range(3):
+        c._sample_nvml()
+    s = c.summary()
+    assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"] and s["source"] == "nvml"
