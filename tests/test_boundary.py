@@ -138,3 +138,19 @@ def test_binding_kernel_list_matches_header():
         text = f.read()
     count = int(re.search(r"FA_KERNEL_COUNT\s*=\s*(\d+)", text).group(1))
     assert count == len(fa.KERNELS)
+
+
+def test_product_path_and_oracle_are_separate():
+    """The package never imports the oracle (no CPU fallback can route through
+    it), and the oracle never loads the CUDA library."""
+    pkg = os.path.join(ROOT, "exact_attention_117_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for name in files:
+            if name.endswith(".py"):
+                text = open(os.path.join(dirpath, name)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", text, re.M), name
+    for name in os.listdir(os.path.join(ROOT, "oracle")):
+        if name.endswith(".py"):
+            text = open(os.path.join(ROOT, "oracle", name)).read()
+            assert "exact_attention_117_b200" not in text and "libfa_b200" not in text, name
+            assert "torch.cuda" not in text and ".cuda(" not in text, name
