@@ -192,3 +192,21 @@ def test_clock_sampler_decodes_nvml_reasons():
     s = c.summary()
     assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
     assert s["reasons"] == ["sw_power_cap"] and s["source"] == "nvml"
+
+
+def test_roofline_entry_for_the_dominant_kernel():
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    totals = {"fwd": 3.0, "bwd_main": 8.0, "bwd_pre": 0.6}
+    per = {"fwd": 0.15, "bwd_main": 0.4, "bwd_pre": 0.03}
+    r = bench.roofline_entry(totals, per, {"fwd": 137.4e9, "bwd_main": 343.6e9},
+                             {"bf16_tflops": 1663.5}, "measured", lambda k: 683e6)
+    assert r["kernel"] == "bwd_main" and r["bound"] == "tensor" and r["traffic"] == 683e6
+    assert abs(r["achieved"] - 343.6e9 / 0.4e-3 / 1e12) < 1e-9
+    assert abs(r["frac"] - r["achieved"] / 1663.5) < 1e-12
+    assert abs(r["frac_of_nominal"] - r["achieved"] / 2250.0) < 1e-12
+    r = bench.roofline_entry({"bwd_pre": 1.0, "fwd": 0.5}, {"bwd_pre": 0.1, "fwd": 0.05},
+                             {"fwd": 1e9}, {"hbm_gbs": 6542.4}, "measured", lambda k: None)
+    assert r["bound"] == "hbm" and r["frac"] is None
