@@ -119,6 +119,8 @@ __device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
 
 // kDq = false (deterministic backward): no dQ MMA and no atomics here; dQ
 // comes from dq_pass_kernel.  dP_{i+1} then only waits for dS_i to be formed.
+constexpr int kHeadGroup = 8;
+
 template <int D, bool kCausal, bool kDq>
 __global__ void __launch_bounds__(384, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -141,8 +143,18 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int j = blockIdx.y;  // key tile; small j (most Q tiles under causal) first
+  // Launch order: heads in groups of kHeadGroup, and within a group key tile
+  // 0 of every head first, then key tile 1, ... (small j = the longest loop
+  // under the causal mask).  The CTAs in flight then share the Q, dO and dQ
+  // accumulator tiles of about kHeadGroup heads, which stay in L2.
+  const int n_kt = np / 128;
+  const int lin = static_cast<int>(blockIdx.x);
+  const int grp = lin / (kHeadGroup * n_kt);
+  const int g_base = grp * kHeadGroup;
+  const int g_size = min(kHeadGroup, static_cast<int>(gridDim.x) / n_kt - g_base);
+  const int g_off = lin - grp * kHeadGroup * n_kt;
+  const int bh = g_base + g_off % g_size;
+  const int j = g_off / g_size;  // key tile
   const int n_q = np / 128;
   const int i0 = kCausal ? j : 0;
   const int n_it = n_q - i0;

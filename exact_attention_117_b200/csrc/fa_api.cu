@@ -222,7 +222,8 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   }
   {
     LaunchTimer timer(st, FA_KERNEL_BWD_MAIN);
-    dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(np / 128));
+    // one CTA per (head, key tile); the kernel maps the linear index to them
+    dim3 grid(static_cast<unsigned>(BH) * static_cast<unsigned>(np / 128));
     fa::bwd_main_kernel<D, C, !kDet><<<grid, L::kThreads, L::kSmemAlloc, st>>>(
         mq, mk, mv, mdo, mdk, mdv, ws.dvec, ws.lse2, ws.dq_acc, N, np, scale, c_exp,
         kWaitLimitNs);
