@@ -109,7 +109,11 @@ fa_status check_common(int B, int H, int N, int d, float scale) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > 0x7fffffffLL) return FA_ERR_SHAPE;
-  if (N > (65535 * 128)) return FA_ERR_SHAPE;  // grid.y limit of the tile axis
+  // kernels that put 128-row tiles on grid.y (the dQ pass) need at most 65535
+  if (N > (65535 * 128)) return FA_ERR_SHAPE;
+  // the backward main kernel runs a linear grid of B*H*ceil(N/128) CTAs, and
+  // the kernels index blocks with 32-bit signed arithmetic
+  if (bh * ((static_cast<long long>(N) + 127) / 128) > 0x7fffffffLL) return FA_ERR_SHAPE;
   if (static_cast<long long>(N) * bh > (1LL << 40)) return FA_ERR_SHAPE;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
   if (!std::isfinite(scale)) return FA_ERR_SCALE;

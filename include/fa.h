@@ -177,6 +177,11 @@ FA_API fa_status fa_bwd_deterministic(const void* q, const void* k, const void* 
  *     order them, e.g. by issuing them on one stream.  Each call rewrites
  *     every part of the array it reads, so leftovers of an earlier call never
  *     leak into its result.
+ *   - The looked-up address is kept for the life of the process.  Do not go
+ *     on using the library on a device after cudaDeviceReset (or any other
+ *     teardown of its primary context) once a call has run there: the kept
+ *     address, like the library's other per-device settings, would belong to
+ *     the destroyed context.
  */
 #define FA_BWD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 FA_API fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,

@@ -29,7 +29,9 @@ Rows are processed in chunks of at most ``row_chunk`` queries purely to bound
 memory (N=16384 would otherwise need a 2 GiB score matrix per slice); every
 row is still the full softmax of that row, with no tiling of the keys.
 
-Pins (tests/test_oracle.py): the page-3 scalar example (50/3, LSE = ln 3),
+Pins (tests/test_oracle.py): the default scale 1/sqrt(d) (exact values,
+brute-force loops with the factor written out, and torch's own default), the
+page-3 scalar example (50/3, LSE = ln 3),
 page-1's running sum, tile-size invariance against the tiled model, causal
 row dependence, the +500 shift, an N=1 closed form, brute-force loops,
 central finite differences for every gradient, and torch's CPU float64

@@ -68,6 +68,15 @@ def test_fwd_rejects_shape(lib, B, H, N):
     assert _fwd(lib, B=B, H=H, N=N) == 2
 
 
+def test_shapes_beyond_the_grid_limits(lib):
+    # B*H*ceil(N/128) above 2^31-1 CTAs: refused before any launch, although
+    # B*H and N are each within their own limits
+    assert _fwd(lib, B=1 << 20, H=1, N=1 << 18) == 2
+    assert _bwd(lib, B=1 << 20, H=1, N=1 << 18, ws_bytes=1 << 62) == 2
+    # 128-row tiles on grid.y: N up to 65535 * 128
+    assert _fwd(lib, N=65535 * 128 + 1) == 2
+
+
 @pytest.mark.parametrize("d", [0, 1, 32, 96, 256])
 def test_fwd_rejects_head_dim(lib, d):
     assert _fwd(lib, d=d) == 3

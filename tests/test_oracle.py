@@ -287,3 +287,63 @@ def test_d_from_output_identity():
         c = attention_backward(q, k, v, do, causal, o_for_d=o + 1e-3)
         assert np.array_equal(c[2], a[2])
         assert np.max(np.abs(c[0] - a[0])) > 1e-6
+
+
+# ------------------------------------------------------------ default scale
+# Page "FlashAttention为什么更快更省显存", opening formula: the scores are
+# Q K^T / sqrt(d_k).  These pins fix the default that every caller leaving
+# ``scale`` out relies on, independently of the oracle's own helper.
+def test_default_scale_values():
+    from oracle import default_scale
+    assert default_scale(64) == 0.125           # 1/sqrt(64), exact in binary
+    assert default_scale(16) == 0.25
+    assert default_scale(4) == 0.5
+    assert abs(default_scale(128) - 0.088388347648318440550) < 3e-17
+    assert abs(default_scale(3) * default_scale(3) * 3 - 1.0) < 1e-15
+
+
+@pytest.mark.parametrize("d", [3, 64])
+@pytest.mark.parametrize("causal", [False, True])
+def test_default_scale_brute_force(d, causal):
+    """scale=None gives the brute-force loops run with 1/sqrt(d) written out."""
+    rng = np.random.default_rng(1000 + d)
+    n = 6
+    q, k, v = _rand(rng, n, d), _rand(rng, n, d), _rand(rng, n, d)
+    o, lse = attention_forward(q, k, v, causal)
+    for i in range(n):
+        keys = range(i + 1) if causal else range(n)
+        sc = [sum(q[i][c] * k[j][c] for c in range(d)) / math.sqrt(d) for j in keys]
+        z = sum(math.exp(x) for x in sc)
+        assert abs(lse[i] - math.log(z)) < 1e-12
+        for c in range(d):
+            ref = sum(math.exp(x) * v[j][c] for x, j in zip(sc, keys)) / z
+            assert abs(o[i][c] - ref) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_default_scale_matches_torch_default(causal):
+    """torch's scaled_dot_product_attention defaults to 1/sqrt(E) on its own;
+    the oracle's forward and backward with scale left out agree with it."""
+    rng = np.random.default_rng(33)
+    n, d = 19, 64
+    q, k, v, do = (_rand(rng, n, d) for _ in range(4))
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(
+        tq[None], tk[None], tv[None], is_causal=causal)[0]
+    to.backward(torch.tensor(do))
+    o, _ = attention_forward(q, k, v, causal)
+    dq, dk, dv = attention_backward(q, k, v, do, causal)
+    assert np.max(np.abs(o - to.detach().numpy())) < 1e-12
+    for g, t in ((dq, tq), (dk, tk), (dv, tv)):
+        assert np.max(np.abs(g - t.grad.numpy())) < 1e-12
+
+
+def test_workload_and_parity_scales():
+    """The seeded workloads and the GPU tests' helper use the same 1/sqrt(d)."""
+    from exact_attention_117_b200.workloads import WORKLOADS
+    from tests.parity_util import default_scale as parity_default_scale
+    assert WORKLOADS["c1"].scale == 0.125 and WORKLOADS["c2"].scale == 0.125
+    assert abs(WORKLOADS["c3"].scale - 0.088388347648318440550) < 3e-17
+    assert WORKLOADS["c4"].scale == WORKLOADS["c3"].scale
+    assert parity_default_scale(64) == 0.125
+    assert abs(parity_default_scale(128) - 0.088388347648318440550) < 3e-17

@@ -36,9 +36,14 @@ def test_noalloc_refuses_problems_larger_than_its_scratch():
 
 @pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_on_two_calls():
-    cases = [Workload("noalloc_a", 2, 4, 1000, 128, seed_base=61),
-             Workload("noalloc_b", 1, 3, 700, 64, seed_base=62)]
-    for w, causal in zip(cases, (True, False)):
+    # the second call's problem fits inside the region the first call wrote, so
+    # it runs over the first call's leftovers; the third repeats the first
+    # shape over the second call's leftovers
+    a = Workload("noalloc_a", 2, 4, 1000, 128, seed_base=61)
+    b = Workload("noalloc_b", 1, 3, 700, 64, seed_base=62)
+    assert fa.workspace_size(b.B, b.H, b.N, b.d) <= fa.workspace_size(a.B, a.H, a.N, a.d)
+    cases = [a, b, Workload("noalloc_a2", 2, 4, 1000, 128, seed_base=63)]
+    for w, causal in zip(cases, (True, False, True)):
         assert fa.workspace_size(w.B, w.H, w.N, w.d) <= fa.NOALLOC_SCRATCH_BYTES
         x = make_inputs(w, "cuda")
         o, lse = fa.forward(x["q"], x["k"], x["v"], causal=causal, scale=w.scale)
