@@ -193,16 +193,22 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
       const uint32_t err = err_k | kErrRoleLoad;
-      mbar_arrive_expect_tx(bar(L::kKvFull), 2 * L::kTile);
-      for (int db = 0; db < kDBlk; ++db) {
-        tma_load_3d(sb + L::kOffK + db * 16384, &tm_k, bar(L::kKvFull), db * 64, j * 128, bh);
-        tma_load_3d(sb + L::kOffV + db * 16384, &tm_v, bar(L::kKvFull), db * 64, j * 128, bh);
+      const int bh_count = static_cast<int>(gridDim.x) / n_kt;
+      // a failed check raises the abort flag; the other roles then give up
+      const bool kv_ok = dbg_check(j * 128 < n && bh < bh_count && i0 + n_it <= n_q, err, abort_flag);
+      if (kv_ok) {
+        mbar_arrive_expect_tx(bar(L::kKvFull), 2 * L::kTile);
+        for (int db = 0; db < kDBlk; ++db) {
+          tma_load_3d(sb + L::kOffK + db * 16384, &tm_k, bar(L::kKvFull), db * 64, j * 128, bh);
+          tma_load_3d(sb + L::kOffV + db * 16384, &tm_v, bar(L::kKvFull), db * 64, j * 128, bh);
+        }
       }
       int nq = 0, ndo = 0;
-      for (int it = 0; it < n_it; ++it) {
+      for (int it = 0; kv_ok && it < n_it; ++it) {
         const int i = i0 + it;
         const int st = it & 1;
-        if (!wait_bounded(bar(L::kQEmpty + st), ((it >> 1) & 1) ^ 1, limit_ns, abort_flag, err))
+        if (!dbg_check(i * 128 < n, err, abort_flag) ||
+            !wait_bounded(bar(L::kQEmpty + st), ((it >> 1) & 1) ^ 1, limit_ns, abort_flag, err))
           break;
         mbar_arrive_expect_tx(bar(L::kQFull + st), L::kTile);
         for (int db = 0; db < kDBlk; ++db)
@@ -218,7 +224,7 @@ __global__ void __launch_bounds__(384, 1)
                       db * 64, i * 128, bh);
         ++ndo;
       }
-      if (*abort_flag) {
+      if (*abort_flag && kv_ok) {
         // copies already issued must land before shared memory is released;
         // with the slab builder's arrival possibly missing, these waits may
         // run to their limit, which only delays the exit
@@ -347,6 +353,8 @@ __global__ void __launch_bounds__(384, 1)
       const int st = it & 1;
       const size_t vrow =
           static_cast<size_t>(bh) * np + static_cast<size_t>(i) * 128 + static_cast<size_t>(lane) * 4;
+      if (!dbg_check(vrow + 4 <= static_cast<size_t>(gridDim.x / n_kt) * np, err, abort_flag))
+        break;
       const float4 l4 = *reinterpret_cast<const float4*>(lse2 + vrow);
       const float4 d4 = *reinterpret_cast<const float4*>(dvec + vrow);
       if (!wait_bounded_warp(bar(L::kQEmpty + st), ((it >> 1) & 1) ^ 1, limit_ns, abort_flag, err))
@@ -390,7 +398,10 @@ __global__ void __launch_bounds__(384, 1)
     const bool key_ok = key < n;
     const uint32_t err = err_k | kErrRoleSoftmax;
     const uint32_t dsrow = sb + L::kOffDS + r * 128;
-    bool ok = true;
+    bool ok = dbg_check(tmem_range_ok(tmem + lane_off + L::kColDP, tmem, 128, L::kTmemCols) &&
+                            tmem_range_ok(tmem + lane_off + L::kColDV, tmem, D, L::kTmemCols) &&
+                            tmem_range_ok(tmem + lane_off + L::kColS, tmem, 128, L::kTmemCols),
+                        err, abort_flag);
     for (int it = 0; it < n_it; ++it) {
       const int i = i0 + it;
       const uint32_t ph = it & 1;
@@ -409,7 +420,7 @@ __global__ void __launch_bounds__(384, 1)
                            *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
         tmem_ld_32x32b_x32(tmem + lane_off + L::kColS + h * 64 + 32,
                            *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-        tmem_wait_ld();
+        tmem_wait_ld_regs(u);
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
           const int c = h * 64 + e;
@@ -446,7 +457,7 @@ __global__ void __launch_bounds__(384, 1)
         const int cc = 2 * h0 + cl;
         uint32_t u[32];
         tmem_ld_32x32b_x32(tmem + lane_off + L::kColDP + cc * 32, u);
-        tmem_wait_ld();
+        tmem_wait_ld_regs(u);
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -474,24 +485,27 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) mbar_arrive(bar(L::kDsReady));
     }
     // ------------------------------------------------------- dK, dV epilogue
-    // dK (scaled) then dV go through the dS^T tile (free once every MMA is
-    // done) as bf16 128-byte-swizzled rows, stored with TMA (rows >= N clip).
+    // Once every MMA is done the dS^T tile and Q stage 0 are free: dK (scaled)
+    // is staged in the first and dV in the second, as bf16 128-byte-swizzled
+    // rows, and both go out with TMA stores issued back to back (rows >= N
+    // clip).  The CTA waits only until the stores have read shared memory.
     if (ok) ok = wait_bounded_warp(bar(L::kDkdvDone), 0, limit_ns, abort_flag, err_k | kErrRoleEpilogue);
     constexpr int kCols = D / 32 / (kDq ? 1 : 2);  // 32-column loads per thread
     const int c_first = kDq ? 0 : h0 * kCols;
+    const uint32_t stage_base[2] = {sb + L::kOffDS, sb + L::kOffQ};
+    if (ok) {
+      tc_fence_after();
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      if (ok) {
-        tc_fence_after();
+      for (int which = 0; which < 2; ++which) {
         const uint32_t col = which == 0 ? L::kColDK : L::kColDV;
         const float mul = which == 0 ? scale : 1.0f;
-        const uint32_t orow = sb + L::kOffDS + r * 128;
+        const uint32_t orow = stage_base[which] + r * 128;
 #pragma unroll
         for (int cl = 0; cl < kCols; ++cl) {
           const int c = c_first + cl;
           uint32_t u[32];
           tmem_ld_32x32b_x32(tmem + lane_off + col + c * 32, u);
-          tmem_wait_ld();
+          tmem_wait_ld_regs(u);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int jj = c * 4 + q;
@@ -506,18 +520,20 @@ __global__ void __launch_bounds__(384, 1)
                                      __uint_as_float(u[8 * q + 7]) * mul));
           }
         }
-        fence_proxy_async_smem();
       }
-      tc_fence_before();
-      named_barrier_sync(1, kWgThreads);  // all compute warps, ok or not
-      if (threadIdx.x == 128 && ok && !*abort_flag) {
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    named_barrier_sync(1, kWgThreads);  // all compute warps, ok or not
+    if (threadIdx.x == 128 && ok && !*abort_flag) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
         const CUtensorMap* map = which == 0 ? &tm_dk : &tm_dv;
         for (int db = 0; db < kDBlk; ++db)
-          tma_store_3d(map, sb + L::kOffDS + db * 16384, db * 64, j * 128, bh);
-        bulk_commit_group();
-        bulk_wait_group_0();  // the staging tile is reused for dV
+          tma_store_3d(map, stage_base[which] + db * 16384, db * 64, j * 128, bh);
       }
-      named_barrier_sync(1, kWgThreads);
+      bulk_commit_group();
+      bulk_wait_group_read_0();  // shared memory stays valid until the stores read it
     }
   } else if (kDq && warp >= 8) {
     // --------------------------------------------------------- dQ read-out
@@ -533,13 +549,16 @@ __global__ void __launch_bounds__(384, 1)
       for (int cc = 0; cc < D / 32; ++cc)
         tmem_ld_32x32b_x32(tmem + lane_off + L::kColDQ + cc * 32,
                            *reinterpret_cast<uint32_t(*)[32]>(&u[cc * 32]));
-      tmem_wait_ld();
+      tmem_wait_ld_regs(u);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::kDqFree));
       // accumulator tile layout [column group of 4][128 rows][4]: lane c's four
       // columns sit next to lane c+1's, so one warp-wide vector add covers 512
       // contiguous bytes (full sectors)
+      if (!dbg_check(static_cast<size_t>(bh) * n_q + i < static_cast<size_t>(gridDim.x), err,
+                     abort_flag))
+        break;
       float* dst = dq_acc + (static_cast<size_t>(bh) * n_q + static_cast<size_t>(i)) * 128 * D +
                    static_cast<size_t>(c) * 4;
 #pragma unroll

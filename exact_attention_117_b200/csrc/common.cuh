@@ -27,7 +27,37 @@ enum : unsigned int {
   kErrRoleDq = 1u << 13,
   kErrAlign = 1u << 14,      // dynamic shared memory base not 1 KiB aligned
   kErrSelfTest = 1u << 15,   // the watchdog self-test kernel gave up (as it must)
+  kErrDebugCheck = 1u << 17, // a bounds check of the FA_DEBUG build failed (see dbg_check)
 };
+
+// ---------------------------------------------------------- debug build
+// Built with -DFA_DEBUG, the kernels check every TMA coordinate, shared-memory
+// destination, TMEM column range and directly indexed global address before
+// using it.  A failed check records kErrDebugCheck and the role's code in the
+// error word, raises the CTA's abort flag and skips the access, so the CTA
+// leaves through the same path as a timed-out wait (no trap, no assert).
+#ifdef FA_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+__device__ __forceinline__ bool dbg_check(bool cond, unsigned int code, volatile int* abort_flag) {
+  if (!kDebugChecks || cond) return true;
+  atomicOr(&g_error_word, kErrDebugCheck | code);
+  *abort_flag = 1;
+  return false;
+}
+
+// TMEM address = (lane << 16) | column; a 32x32b access of `cols` columns by
+// a warp of a 4-warp group must stay inside the `alloc` allocated columns.
+__device__ __forceinline__ bool tmem_range_ok(uint32_t addr, uint32_t base, uint32_t cols,
+                                              uint32_t alloc) {
+  const uint32_t col = (addr & 0xffffu) - (base & 0xffffu);
+  const uint32_t lane = (addr >> 16) - (base >> 16);
+  return (addr & 0xffffu) >= (base & 0xffffu) && col + cols <= alloc && lane < 128u &&
+         (lane & 31u) == 0u;
+}
 
 // Second bound on every wait, in case the global timer were ever to stand
 // still: far above any legitimate wait of these kernels.
@@ -72,6 +102,31 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
       atomicOr(&g_error_word, kErrRoleDrain);
       return;
     }
+  }
+}
+
+// ------------------------------------------------------ work distribution
+// Persistent kernels launch about one CTA per SM; each CTA takes its first
+// work item from blockIdx.x and every further one from a per-launch counter
+// (one atomicAdd each), so items (ordered longest first) go to whichever CTA
+// frees up first.  The counters live here: a launch uses slot (per-device
+// launch sequence number mod kSchedSlots), finds it at zero, and the last of
+// its CTAs to finish sets it back to zero -- also after a timed-out wait,
+// since every CTA leaves through the same exit -- so a replay of the same
+// launch (a captured CUDA graph) starts from zero too.  Two launches share a
+// slot only kSchedSlots launches apart.
+constexpr int kSchedSlots = 1 << 14;
+__device__ unsigned int g_sched_next[kSchedSlots];
+__device__ unsigned int g_sched_done[kSchedSlots];
+
+// Called once per CTA by one thread after all of the CTA's work: the last CTA
+// of the launch clears the slot for the next launch that uses it.
+__device__ __forceinline__ void sched_finish(uint32_t slot) {
+  __threadfence();
+  const unsigned int done = atomicAdd(&g_sched_done[slot], 1u);
+  if (done == gridDim.x - 1) {
+    atomicExch(&g_sched_next[slot], 0u);
+    atomicExch(&g_sched_done[slot], 0u);
   }
 }
 

@@ -111,15 +111,20 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
       const uint32_t err = err_k | kErrRoleLoad;
-      mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTile);
-      for (int db = 0; db < kDBlk; ++db) {
-        tma_load_3d(sb + L::kOffQ + db * 16384, &tm_q, bar(L::kQFull), db * 64, i * 128, bh);
-        tma_load_3d(sb + L::kOffDO + db * 16384, &tm_do, bar(L::kQFull), db * 64, i * 128, bh);
+      // a failed check raises the abort flag; the other roles then give up
+      const bool q_ok = dbg_check(i * 128 < n && n_kv * 128 <= np, err, abort_flag);
+      if (q_ok) {
+        mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTile);
+        for (int db = 0; db < kDBlk; ++db) {
+          tma_load_3d(sb + L::kOffQ + db * 16384, &tm_q, bar(L::kQFull), db * 64, i * 128, bh);
+          tma_load_3d(sb + L::kOffDO + db * 16384, &tm_do, bar(L::kQFull), db * 64, i * 128, bh);
+        }
       }
       int nk = 0, nv = 0;
-      for (int j = 0; j < n_kv; ++j) {
+      for (int j = 0; q_ok && j < n_kv; ++j) {
         const int sk = j % KS, sv = j % VS;
-        if (!wait_bounded(bar(L::kKEmpty + sk), ((j / KS) & 1) ^ 1, limit_ns, abort_flag, err))
+        if (!dbg_check(j * 128 < n, err, abort_flag) ||
+            !wait_bounded(bar(L::kKEmpty + sk), ((j / KS) & 1) ^ 1, limit_ns, abort_flag, err))
           break;
         mbar_arrive_expect_tx(bar(L::kKFull + sk), L::kTile);
         for (int db = 0; db < kDBlk; ++db)
@@ -134,7 +139,7 @@ __global__ void __launch_bounds__(384, 1)
                       db * 64, j * 128, bh);
         ++nv;
       }
-      if (*abort_flag) {
+      if (*abort_flag && q_ok) {
         drain_wait(bar(L::kQFull), 0, limit_ns);
         for (int j = (nk > KS ? nk - KS : 0); j < nk; ++j)
           drain_wait(bar(L::kKFull + j % KS), (j / KS) & 1, limit_ns);
@@ -245,7 +250,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t u[64];
         tmem_ld_32x32b_x32(xa, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
         tmem_ld_32x32b_x32(xa + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-        tmem_wait_ld();
+        tmem_wait_ld_regs(u);
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
           float p0 = ex2_approx(fmaf(__uint_as_float(u[e]), c_exp, neg_l2));
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t ya = tmem + lane_off + L::kColDP + cb;
         tmem_ld_32x32b_x32(ya, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
         tmem_ld_32x32b_x32(ya + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-        tmem_wait_ld();
+        tmem_wait_ld_regs(u);
         uint32_t w[32];
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(384, 1)
         const int c0 = wg * (D / 2) + c * 32;  // first dQ column of this load
         uint32_t u[32];
         tmem_ld_32x32b_x32(tmem + lane_off + L::kColDQ + c0, u);
-        tmem_wait_ld();
+        tmem_wait_ld_regs(u);
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int jj = c0 / 8 + g;  // 16-byte chunk of the output row
@@ -315,7 +320,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int db = 0; db < kDBlk; ++db)
         tma_store_3d(&tm_dq, sb + L::kOffQ + db * 16384, db * 64, i * 128, bh);
       bulk_commit_group();
-      bulk_wait_group_0();
+      bulk_wait_group_read_0();
     }
   }
 

@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -162,27 +163,42 @@ BwdWorkspace bwd_workspace_layout(void* base, int B, int H, int N, int d) {
   return w;
 }
 
+// Per-device launch sequence numbers: a persistent kernel's launch takes work
+// counter slot (sequence mod kSchedSlots) (see common.cuh).
+std::atomic<uint32_t> g_launch_seq[kMaxDevices];
+
+uint32_t next_sched_slot(int dev) {
+  return g_launch_seq[dev].fetch_add(1u) & static_cast<uint32_t>(fa::kSchedSlots - 1);
+}
+
 template <int D, bool C, bool kSplit>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const CUtensorMap& mo, float* lse, int BH, int N, float scale_log2,
-                     cudaStream_t st, int num_splits = 1, float* part_o = nullptr,
-                     float* part_lse = nullptr) {
+                     void* o, float* lse, int BH, int N, float scale_log2, cudaStream_t st,
+                     int num_splits = 1, float* part_o = nullptr, float* part_lse = nullptr) {
   using L = fa::FwdLayout<D>;
   static bool attr_set[kMaxDevices] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return FA_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
   if (!attr_set[dev]) {
     if (!set_smem(fa::fwd_kernel<D, C, kSplit>, L::kSmemAlloc)) return FA_ERR_CUDA;
     attr_set[dev] = true;
   }
   const int q_tiles = (N + L::kBM - 1) / L::kBM;
-  // 2 Q tiles per CTA; one CTA per split of the key range in split mode
-  dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>((q_tiles + 1) / 2),
-            static_cast<unsigned>(kSplit ? num_splits : 1));
+  const int pairs = (q_tiles + 1) / 2;
+  // Work items: (head, pair of Q tiles[, split]).  Up to 48 heads form one
+  // launch-order group; more heads go in groups of 32, so that about
+  // 148 / 32 busy CTAs per head share its K/V tiles in L2.
+  const int head_group = BH <= 48 ? BH : 32;
+  const long long items = static_cast<long long>(BH) * pairs * (kSplit ? num_splits : 1);
+  if (items > 0x7fffffffLL) return FA_ERR_SHAPE;
+  const int n_items = static_cast<int>(items);
+  const int grid = std::min(n_items, sm_count(dev));  // persistent: one CTA per SM
+  const uint32_t slot = next_sched_slot(dev);
   {
     LaunchTimer timer(st, FA_KERNEL_FWD);
     fa::fwd_kernel<D, C, kSplit><<<grid, 384, L::kSmemAlloc, st>>>(
-        mq, mk, mv, mo, lse, N, scale_log2, kWaitLimitNs, num_splits, part_o, part_lse);
+        mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, N, BH, scale_log2, kWaitLimitNs,
+        num_splits, part_o, part_lse, head_group, n_items, slot);
   }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -335,17 +351,17 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_ALIGN;
   const int bh = B * H;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv;
   if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
-      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mo, o, d, N, bh, 128))
+      !encode_bf16_3d(&mv, v, d, N, bh, 128))
     return FA_ERR_CUDA;
   const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
-    return causal ? launch_fwd<64, true, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
-                  : launch_fwd<64, false, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
-  return causal ? launch_fwd<128, true, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
-                : launch_fwd<128, false, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
+    return causal ? launch_fwd<64, true, false>(mq, mk, mv, o, lse, bh, N, scale_log2, s)
+                  : launch_fwd<64, false, false>(mq, mk, mv, o, lse, bh, N, scale_log2, s);
+  return causal ? launch_fwd<128, true, false>(mq, mk, mv, o, lse, bh, N, scale_log2, s)
+                : launch_fwd<128, false, false>(mq, mk, mv, o, lse, bh, N, scale_log2, s);
 }
 
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits) {
@@ -380,14 +396,14 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   fa_status r;
   if (d == 64)
-    r = causal ? launch_fwd<64, true, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s, num_splits,
-                                            part_o, part_lse)
-               : launch_fwd<64, false, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
+    r = causal ? launch_fwd<64, true, true>(mq, mk, mv, nullptr, lse, bh, N, scale_log2, s,
+                                            num_splits, part_o, part_lse)
+               : launch_fwd<64, false, true>(mq, mk, mv, nullptr, lse, bh, N, scale_log2, s,
                                              num_splits, part_o, part_lse);
   else
-    r = causal ? launch_fwd<128, true, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
+    r = causal ? launch_fwd<128, true, true>(mq, mk, mv, nullptr, lse, bh, N, scale_log2, s,
                                              num_splits, part_o, part_lse)
-               : launch_fwd<128, false, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
+               : launch_fwd<128, false, true>(mq, mk, mv, nullptr, lse, bh, N, scale_log2, s,
                                               num_splits, part_o, part_lse);
   if (r != FA_OK) return r;
   {

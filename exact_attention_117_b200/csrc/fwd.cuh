@@ -9,12 +9,25 @@
 // accumulates; O / l and the row logsumexp are written once at the end.  No
 // N x N tensor ever reaches global memory.
 //
-// One CTA owns TWO consecutive 128-row Q tiles of one (batch, head) and runs
-// them ping-pong: while the softmax warps of one tile work on its scores, the
+// A work item is TWO consecutive 128-row Q tiles of one (batch, head) (and,
+// for the split-KV forward, one range of key tiles); the CTA runs the two
+// tiles ping-pong: while the softmax warps of one tile work on its scores, the
 // tensor core computes P V and the next S = Q K^T of the other tile.
 //
+// The kernel is persistent: about one CTA per SM, each taking items until
+// none are left (the first from blockIdx.x, the rest from a per-launch work
+// counter, longest items first).  The K/V ring and every barrier phase run on
+// across items, so the next item's Q and first K/V tiles load, and its first
+// scores are computed, while the previous item's last tiles and epilogue are
+// still in flight; the epilogue writes O straight from registers to global
+// memory, so it holds no shared memory the next item needs.
+//
 // Warp roles (384 threads):
-//   warp 0      : TMA producer (both Q tiles once, then K_j / V_j rings)
+//   warp 0      : TMA producer (an item's two Q tiles, then its K_j / V_j) and
+//                 scheduler: once an item's loads are issued it takes the next
+//                 item from the counter and publishes it in a two-slot ring
+//                 that the other roles read (an item is claimed only when this
+//                 CTA is about to load it, so the counter keeps the balance)
 //   warp 1      : TMEM allocator and tcgen05.mma issuer
 //   warps 2-3   : idle
 //   warps 4-7   : softmax of Q tile 0, one thread per query row
@@ -60,46 +73,94 @@ struct FwdLayout {
   static constexpr int kOffK = 2 * kTile;
   static constexpr int kOffV = kOffK + kStages * kTile;
   static constexpr int kOffBar = kOffV + kStages * kTile;
-  static constexpr int kBarArea = 256;
+  static constexpr int kBarArea = 512;
   static constexpr int kBytes = kOffBar + kBarArea;
   static constexpr int kSmemAlloc = kBytes + 1024;  // slack to align the base to 1 KiB
   // barrier indices
   static constexpr int kQFull = 0;
-  static constexpr int kKFull = 1;
+  static constexpr int kQEmpty = 1;
+  static constexpr int kKFull = 2;
   static constexpr int kKEmpty = kKFull + kStages;
   static constexpr int kVFull = kKEmpty + kStages;
   static constexpr int kVEmpty = kVFull + kStages;
   static constexpr int kSFull = kVEmpty + kStages;  // [2]
   static constexpr int kPFull = kSFull + 2;         // [2]
   static constexpr int kOFinal = kPFull + 2;        // [2]
-  static constexpr int kDrain = kOFinal + 2;
+  static constexpr int kItemFull = kOFinal + 2;     // [2]
+  static constexpr int kItemEmpty = kItemFull + 2;  // [2]
+  static constexpr int kDrain = kItemEmpty + 2;
   static constexpr int kNumBars = kDrain + 1;
   static constexpr int kOffSlot = kOffBar + 8 * kNumBars;  // TMEM base address
   static constexpr int kOffAbort = kOffSlot + 4;
-  static_assert(kOffAbort + 4 <= kOffBar + kBarArea, "barrier area too small");
+  static constexpr int kOffItems = kOffAbort + 4;  // [2] item ring
+  static_assert(kOffItems + 8 <= kOffBar + kBarArea, "barrier area too small");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128;
   static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
-  static constexpr float kRescaleThreshold = 8.0f;  // base-2 units
+  static constexpr float kRescaleThreshold = 8.0f;    // base-2 units
+  static constexpr float kSpecRedoThreshold = 20.0f;  // base-2 units, speculative tiles
   static constexpr uint32_t kLaunchRegs = 168;      // 65536 / 384, rounded down to 8
   static constexpr uint32_t kRegsOther = 80;
   static constexpr uint32_t kRegsSoftmax = 200;
   static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= 384 * kLaunchRegs, "register split");
+  // arrivals that free an item ring slot: MMA warp, 8 softmax warps
+  static constexpr uint32_t kItemReaders = 9;
 };
 
-// kSplit: the CTA covers only the key tiles of split blockIdx.z (a contiguous
-// range of ceil(n_kv / num_splits) tiles) and writes, instead of O and LSE,
-// fp32 partial results: O_s = u_s / l_s in the tile layout [D/4 column
-// groups][128 rows][4] of part_o, and LSE_s = m_s + log2 l_s (base 2) in
-// part_lse; a split that sees no key of a row writes O_s = 0, LSE_s = -inf.
+// One work item: Q tiles qt0 and qt1 of slice bh, key tiles [kb, kb + n1).
+struct FwdItem {
+  int bh, qt0, qt1, kb, n0, n1, split;
+  bool single;  // odd tile count: only qt1 (== qt0) is real, tile 0 idles
+};
+
+// Item order: heads in groups of head_group; within a group the pairs with
+// the most key tiles come first, every head of the group at each pair; the
+// splits of one (head, pair) are consecutive.  The CTAs busy at any time then
+// read the K/V of a bounded set of heads, which stays in L2.
+template <bool kCausal, bool kSplit>
+__device__ __forceinline__ FwdItem fwd_item(int item, int n_kv_all, int bh_count, int head_group,
+                                            int num_splits) {
+  FwdItem w;
+  const int n_pairs = (n_kv_all + 1) / 2;
+  w.split = kSplit ? item % num_splits : 0;
+  const int lin = kSplit ? item / num_splits : item;
+  const int grp = lin / (head_group * n_pairs);
+  const int g_base = grp * head_group;
+  const int g_size = min(head_group, bh_count - g_base);
+  const int g_off = lin - grp * head_group * n_pairs;
+  const int pair = n_pairs - 1 - g_off / g_size;
+  w.bh = g_base + g_off % g_size;
+  w.single = 2 * pair + 1 >= n_kv_all;
+  w.qt0 = 2 * pair;
+  w.qt1 = w.single ? 2 * pair : 2 * pair + 1;
+  int kb = 0, ke = n_kv_all;
+  if (kSplit) {
+    const int chunk = (n_kv_all + num_splits - 1) / num_splits;
+    kb = w.split * chunk;
+    ke = min(kb + chunk, n_kv_all);
+  }
+  const int end0 = kCausal ? min(w.qt0 + 1, n_kv_all) : n_kv_all;
+  const int end1 = kCausal ? min(w.qt1 + 1, n_kv_all) : n_kv_all;
+  w.kb = kb;
+  w.n0 = w.single ? 0 : max(0, min(ke, end0) - kb);
+  w.n1 = max(0, min(ke, end1) - kb);  // n1 >= n0; a split may have 0
+  return w;
+}
+
+// kSplit: an item covers only the key tiles of its split (a contiguous range
+// of ceil(n_kv / num_splits) tiles) and writes, instead of O and LSE, fp32
+// partial results: O_s = u_s / l_s in the tile layout [D/4 column groups][128
+// rows][4] of part_o, and LSE_s = m_s + log2 l_s (base 2) in part_lse; a split
+// that sees no key of a row writes O_s = 0, LSE_s = -inf.
 // splitkv_combine_kernel merges the splits.
 template <int D, bool kCausal, bool kSplit>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-               float* __restrict__ lse_out, int n, float scale_log2, uint64_t limit_ns,
-               int num_splits, float* __restrict__ part_o, float* __restrict__ part_lse) {
+               const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ o_out,
+               float* __restrict__ lse_out, int n, int bh_count, float scale_log2,
+               uint64_t limit_ns, int num_splits, float* __restrict__ part_o,
+               float* __restrict__ part_lse, int head_group, int n_items, uint32_t sched_slot) {
   using L = FwdLayout<D>;
   constexpr int S = L::kStages;
   constexpr int kDBlk = D / 64;  // 128-byte swizzle blocks per tile row
@@ -110,31 +171,21 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sb + L::kOffBar + 8u * static_cast<uint32_t>(i); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
+  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::kOffItems);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffSlot);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int pair = static_cast<int>(gridDim.y) - 1 - static_cast<int>(blockIdx.y);  // heavy first
   const int n_kv_all = (n + L::kBN - 1) / L::kBN;  // also the number of Q tiles (Nq = Nk)
-  const int qt0 = 2 * pair, qt1 = 2 * pair + 1;
-  // key tiles [kb, ke) of this CTA: all of them, or this split's share
-  int kb = 0, ke = n_kv_all;
-  if (kSplit) {
-    const int chunk = (n_kv_all + num_splits - 1) / num_splits;
-    kb = static_cast<int>(blockIdx.z) * chunk;
-    ke = min(kb + chunk, n_kv_all);
-  }
-  const int end0 = kCausal ? min(qt0 + 1, n_kv_all) : n_kv_all;  // causal end, Q tile 0
-  const int end1 = kCausal ? min(qt1 + 1, n_kv_all) : n_kv_all;  // causal end, Q tile 1
-  // key tiles each Q tile processes here, from kb on (n1 >= n0; a split may have 0)
-  const int n0 = max(0, min(ke, end0) - kb);
-  const int n1 = max(0, min(ke, end1) - kb);
   const unsigned int err_fwd = kErrFwd;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < L::kNumBars; ++b)
-      mbar_init(bar(b), (b == L::kPFull || b == L::kPFull + 1) ? 4u : 1u);
+    for (int b = 0; b < L::kNumBars; ++b) {
+      uint32_t cnt = 1;
+      if (b == L::kPFull || b == L::kPFull + 1) cnt = 4;
+      if (b == L::kItemEmpty || b == L::kItemEmpty + 1) cnt = L::kItemReaders;
+      mbar_init(bar(b), cnt);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -148,118 +199,216 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Item k of this CTA from the ring (warp-uniform); false if the wait gave
+  // up.  Every reader arrives once per item on the slot's empty barrier
+  // (lane 0 of each reading warp).
+  auto read_item = [&](int k, int& item, unsigned int err) -> bool {
+    if (!wait_bounded_warp(bar(L::kItemFull + (k & 1)), (k >> 1) & 1, limit_ns, abort_flag, err))
+      return false;
+    item = item_ring[k & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(L::kItemEmpty + (k & 1)));
+    return true;
+  };
+
   // Registers: the block launches with 168 per thread (384 x 168 = 64512).
-  // Load / MMA / idle warps drop to 80, the two softmax warp groups rise to
-  // 200: 128 x 80 + 256 x 200 = 61440 <= 64512.
+  // Load / MMA / idle warps drop to 80, the two softmax warp groups rise
+  // to 200: 128 x 80 + 256 x 200 = 61440 <= 64512.
   if (warp < 4) {
     setmaxnreg_dec<L::kRegsOther>();
     if (warp == 0) {
-      // ------------------------------------------------------------ producer
+      // --------------------------------------------------- producer, scheduler
+      const uint32_t err = err_fwd | kErrRoleLoad;
       if (lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-        tma_prefetch_desc(&tm_o);
-        const uint32_t err = err_fwd | kErrRoleLoad;
-        int nk = 0, nv = 0;
-        if (n1 > 0) mbar_arrive_expect_tx(bar(L::kQFull), 2 * L::kTile);
-        for (int db = 0; n1 > 0 && db < kDBlk; ++db) {
-          tma_load_3d(sb + L::kOffQ0 + db * 16384, &tm_q, bar(L::kQFull), db * 64, qt0 * L::kBM, bh);
-          tma_load_3d(sb + L::kOffQ1 + db * 16384, &tm_q, bar(L::kQFull), db * 64, qt1 * L::kBM, bh);
+      }
+      int g_kv = 0;   // K/V tiles issued so far (ring position)
+      int q_cnt = 0;  // items whose Q tiles were loaded
+      bool q_pending = false;
+      int nk = 0, nv = 0;  // K and V tiles issued
+      // publishes item k (or -1: no more work) in ring slot k & 1 once every
+      // reader has taken item k - 2 from it
+      auto publish = [&](int k, int item) -> bool {
+        bool ok = true;
+        if (lane == 0) {
+          ok = wait_bounded(bar(L::kItemEmpty + (k & 1)), ((k >> 1) & 1) ^ 1, limit_ns, abort_flag,
+                            err);
+          if (ok) {
+            item_ring[k & 1] = item;
+            mbar_arrive(bar(L::kItemFull + (k & 1)));  // release: readers acquire the slot
+          }
         }
-        for (int jj = 0; jj < n1; ++jj) {
-          const int j = kb + jj;  // key tile
-          const int s = jj % S;
-          const uint32_t ph = (jj / S) & 1;
-          if (!wait_bounded(bar(L::kKEmpty + s), ph ^ 1, limit_ns, abort_flag, err)) break;
-          mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTile);
-          for (int db = 0; db < kDBlk; ++db)
-            tma_load_3d(sb + L::kOffK + s * L::kTile + db * 16384, &tm_k, bar(L::kKFull + s),
-                        db * 64, j * L::kBN, bh);
-          ++nk;
-          if (!wait_bounded(bar(L::kVEmpty + s), ph ^ 1, limit_ns, abort_flag, err)) break;
-          mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTile);
-          for (int db = 0; db < kDBlk; ++db)
-            tma_load_3d(sb + L::kOffV + s * L::kTile + db * 16384, &tm_v, bar(L::kVFull + s),
-                        db * 64, j * L::kBN, bh);
-          ++nv;
+        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      };
+      int item = static_cast<int>(blockIdx.x);
+      for (int k = 0; publish(k, item); ++k) {
+        if (item < 0) break;
+        const FwdItem w = fwd_item<kCausal, kSplit>(item, n_kv_all, bh_count, head_group, num_splits);
+        if (lane == 0 && w.n1 > 0) {
+          bool ok = true;
+          // the Q buffers are free once the previous item's last S MMA is done
+          if (q_cnt > 0)
+            ok = wait_bounded(bar(L::kQEmpty), (q_cnt - 1) & 1, limit_ns, abort_flag, err);
+          ok = ok && dbg_check(w.qt0 >= 0 && w.qt1 * L::kBM < n && w.bh >= 0 && w.bh < bh_count &&
+                                   w.kb >= 0 && w.kb + w.n1 <= n_kv_all,
+                               err, abort_flag);
+          if (ok) {
+            mbar_arrive_expect_tx(bar(L::kQFull), (w.single ? 1 : 2) * L::kTile);
+            for (int db = 0; db < kDBlk; ++db) {
+              if (!w.single)
+                tma_load_3d(sb + L::kOffQ0 + db * 16384, &tm_q, bar(L::kQFull), db * 64,
+                            w.qt0 * L::kBM, w.bh);
+              tma_load_3d(sb + L::kOffQ1 + db * 16384, &tm_q, bar(L::kQFull), db * 64,
+                          w.qt1 * L::kBM, w.bh);
+            }
+            q_pending = true;
+          }
+          for (int jj = 0; ok && jj < w.n1; ++jj) {
+            const int gi = g_kv + jj;
+            const int j = w.kb + jj;  // key tile
+            const int s = gi % S;
+            const uint32_t ph = (gi / S) & 1;
+            if (!dbg_check(j * L::kBN < n && L::kOffV + (s + 1) * L::kTile <= L::kOffBar, err,
+                           abort_flag) ||
+                !wait_bounded(bar(L::kKEmpty + s), ph ^ 1, limit_ns, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(L::kKFull + s), L::kTile);
+            for (int db = 0; db < kDBlk; ++db)
+              tma_load_3d(sb + L::kOffK + s * L::kTile + db * 16384, &tm_k, bar(L::kKFull + s),
+                          db * 64, j * L::kBN, w.bh);
+            ++nk;
+            if (!wait_bounded(bar(L::kVEmpty + s), ph ^ 1, limit_ns, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(L::kVFull + s), L::kTile);
+            for (int db = 0; db < kDBlk; ++db)
+              tma_load_3d(sb + L::kOffV + s * L::kTile + db * 16384, &tm_v, bar(L::kVFull + s),
+                          db * 64, j * L::kBN, w.bh);
+            ++nv;
+          }
+          if (!ok) item = -2;  // leave the item loop (after the drain below)
         }
-        if (*abort_flag && n1 > 0) {
-          // let every copy already issued land before shared memory is released
-          drain_wait(bar(L::kQFull), 0, limit_ns);
-          for (int j = (nk > S ? nk - S : 0); j < nk; ++j)
-            drain_wait(bar(L::kKFull + j % S), (j / S) & 1, limit_ns);
-          for (int j = (nv > S ? nv - S : 0); j < nv; ++j)
-            drain_wait(bar(L::kVFull + j % S), (j / S) & 1, limit_ns);
+        if (__shfl_sync(0xffffffffu, item, 0) == -2) break;
+        if (w.n1 > 0) {
+          ++q_cnt;
+          g_kv += w.n1;
         }
+        // claim the next item now that this one's loads are all issued
+        unsigned int f = 0;
+        if (lane == 0) f = atomicAdd(&g_sched_next[sched_slot], 1u);
+        f = __shfl_sync(0xffffffffu, f, 0);
+        item = f >= static_cast<unsigned int>(n_items) - gridDim.x ? -1
+                                                                    : static_cast<int>(gridDim.x + f);
+      }
+      if (lane == 0 && *abort_flag && q_pending) {
+        // let every copy already issued land before shared memory is released
+        drain_wait(bar(L::kQFull), (q_cnt - 1) & 1, limit_ns);
+        for (int j = (nk > S ? nk - S : 0); j < nk; ++j)
+          drain_wait(bar(L::kKFull + j % S), (j / S) & 1, limit_ns);
+        for (int j = (nv > S ? nv - S : 0); j < nv; ++j)
+          drain_wait(bar(L::kVFull + j % S), (j / S) & 1, limit_ns);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
       // the whole warp runs this loop; the MMA and commit wrappers elect one lane
-      {
-        constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t id_o = idesc_bf16_f32(128, D, false, true);
-        const uint32_t err = err_fwd | kErrRoleMma;
-        auto issue_s = [&](int t, int jj) {  // S_t = Q_t K_j^T, key tile j = kb + jj
-          const uint32_t qa = sb + (t ? L::kOffQ1 : L::kOffQ0);
-          const uint32_t ka = sb + L::kOffK + (jj % S) * L::kTile;
-          const uint32_t d_tmem = tmem + (t ? L::kColS1 : L::kColS0);
-  #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(d_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), id_s,
-                        kk > 0 ? 1u : 0u);
-          }
-          tc_commit(bar(L::kSFull + t));
-        };
-        auto issue_pv = [&](int t, int jj) {  // O_t += P_t V_j, P_t from TMEM
-          const uint32_t va = sb + L::kOffV + (jj % S) * L::kTile;
-          const uint32_t d_tmem = tmem + (t ? L::kColO1 : L::kColO0);
-          const uint32_t a_tmem = tmem + (t ? L::kColS1 : L::kColS0);
-  #pragma unroll
-          for (int kk = 0; kk < L::kBN / 16; ++kk)
-            mma_bf16_ts(d_tmem, a_tmem + kk * 8, sw128_desc(va + kk * 2048, 16384, 1024), id_o,
-                        (jj > 0 || kk > 0) ? 1u : 0u);
-        };
-        bool ok = n1 > 0 && wait_bounded_warp(bar(L::kQFull), 0, limit_ns, abort_flag, err) &&
-                  wait_bounded_warp(bar(L::kKFull), 0, limit_ns, abort_flag, err);
-        if (ok) {
-          tc_fence_after();
-          if (n0 > 0) issue_s(0, 0);
-          issue_s(1, 0);
-          tc_commit(bar(L::kKEmpty));
+      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t err = err_fwd | kErrRoleMma;
+      auto issue_s = [&](int t, int gi) {  // S_t = Q_t K^T, K from ring position gi
+        const uint32_t qa = sb + (t ? L::kOffQ1 : L::kOffQ0);
+        const uint32_t ka = sb + L::kOffK + (gi % S) * L::kTile;
+        const uint32_t d_tmem = tmem + (t ? L::kColS1 : L::kColS0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_bf16_ss(d_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), id_s,
+                      kk > 0 ? 1u : 0u);
         }
-        for (int jj = 0; ok && jj < n1; ++jj) {
-          const int s = jj % S;
-          if (!wait_bounded_warp(bar(L::kVFull + s), (jj / S) & 1, limit_ns, abort_flag, err)) break;
+        tc_commit(bar(L::kSFull + t));
+      };
+      auto issue_pv = [&](int t, int gi, bool first) {  // O_t (+)= P_t V, P_t from TMEM
+        const uint32_t va = sb + L::kOffV + (gi % S) * L::kTile;
+        const uint32_t d_tmem = tmem + (t ? L::kColO1 : L::kColO0);
+        const uint32_t a_tmem = tmem + (t ? L::kColS1 : L::kColS0);
+#pragma unroll
+        for (int kk = 0; kk < L::kBN / 16; ++kk)
+          mma_bf16_ts(d_tmem, a_tmem + kk * 8, sw128_desc(va + kk * 2048, 16384, 1024), id_o,
+                      (!first || kk > 0) ? 1u : 0u);
+      };
+      int g_kv = 0, q_cnt = 0, p0 = 0, p1 = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        int item;
+        if (!read_item(k, item, err)) break;
+        if (item < 0) break;
+        const FwdItem w = fwd_item<kCausal, kSplit>(item, n_kv_all, bh_count, head_group, num_splits);
+        const int n0 = w.n0, n1 = w.n1;
+        if (n1 == 0) continue;
+        ok = dbg_check(tmem_range_ok(tmem + L::kColO1, tmem, D, L::kTmemCols) &&
+                           tmem_range_ok(tmem + L::kColS1, tmem, 128, L::kTmemCols),
+                       err, abort_flag) &&
+             wait_bounded_warp(bar(L::kQFull), q_cnt & 1, limit_ns, abort_flag, err) &&
+             wait_bounded_warp(bar(L::kKFull + g_kv % S), (g_kv / S) & 1, limit_ns, abort_flag, err);
+        ++q_cnt;
+        if (!ok) break;
+        tc_fence_after();
+        if (n0 > 0) issue_s(0, g_kv);
+        issue_s(1, g_kv);
+        tc_commit(bar(L::kKEmpty + g_kv % S));
+        if (n1 == 1) tc_commit(bar(L::kQEmpty));  // the item's last S reads of Q are issued
+        for (int jj = 0; jj < n1; ++jj) {
+          const int gi = g_kv + jj;
+          const int s = gi % S;
+          if (!wait_bounded_warp(bar(L::kVFull + s), (gi / S) & 1, limit_ns, abort_flag, err)) {
+            ok = false;
+            break;
+          }
           if (jj < n0) {
-            if (!wait_bounded_warp(bar(L::kPFull + 0), jj & 1, limit_ns, abort_flag, err)) break;
+            if (!wait_bounded_warp(bar(L::kPFull + 0), p0 & 1, limit_ns, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            ++p0;
             tc_fence_after();
-            issue_pv(0, jj);
+            issue_pv(0, gi, jj == 0);
             if (jj == n0 - 1) tc_commit(bar(L::kOFinal + 0));
           }
           const bool next = jj + 1 < n1;
-          const int s1 = (jj + 1) % S;
+          const int s1 = (gi + 1) % S;
           if (next) {
-            if (!wait_bounded_warp(bar(L::kKFull + s1), ((jj + 1) / S) & 1, limit_ns, abort_flag, err))
+            if (!wait_bounded_warp(bar(L::kKFull + s1), ((gi + 1) / S) & 1, limit_ns, abort_flag,
+                                   err)) {
+              ok = false;
               break;
+            }
             tc_fence_after();
-            if (jj + 1 < n0) issue_s(0, jj + 1);
+            if (jj + 1 < n0) issue_s(0, gi + 1);
           }
-          if (!wait_bounded_warp(bar(L::kPFull + 1), jj & 1, limit_ns, abort_flag, err)) break;
+          if (!wait_bounded_warp(bar(L::kPFull + 1), p1 & 1, limit_ns, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          ++p1;
           tc_fence_after();
-          issue_pv(1, jj);
+          issue_pv(1, gi, jj == 0);
           if (jj == n1 - 1) tc_commit(bar(L::kOFinal + 1));
           tc_commit(bar(L::kVEmpty + s));
           if (next) {
-            issue_s(1, jj + 1);
+            issue_s(1, gi + 1);
             tc_commit(bar(L::kKEmpty + s1));
+            if (jj + 2 == n1) tc_commit(bar(L::kQEmpty));  // last S reads of Q issued
           }
         }
-        // every MMA issued above must finish before TMEM / smem are released
-        tc_commit(bar(L::kDrain));
-        drain_wait(bar(L::kDrain), 0, limit_ns);
+        g_kv += n1;
       }
+      // every MMA issued above must finish before TMEM / smem are released
+      tc_commit(bar(L::kDrain));
+      drain_wait(bar(L::kDrain), 0, limit_ns);
       __syncwarp();
     }
   } else {
@@ -267,196 +416,284 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------- softmax / epilogue
     const int t = (warp >= 8) ? 1 : 0;         // which Q tile
     const int r = threadIdx.x - 128 - 128 * t;  // row inside the tile == TMEM lane
-    const int qt = qt0 + t;
-    const int n_t = t ? n1 : n0;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + (t ? L::kColS1 : L::kColS0);
     const uint32_t o_addr = tmem + lane_off + (t ? L::kColO1 : L::kColO0);
     const uint32_t err = err_fwd | kErrRoleSoftmax;
     const bool neg_scale = scale_log2 < 0.f;
     const uint32_t masked_bits = __float_as_uint(neg_scale ? INFINITY : -INFINITY);
-    float m_run = -INFINITY;  // running (possibly stale) max of scale*log2(e)*s
-    float l_run = 0.f;        // running sum of 2^(x - m_run)
+    int s_cnt = 0, of_cnt = 0;  // S tiles and final O of this tile seen so far
     bool ok = true;
-    for (int jj = 0; jj < n_t; ++jj) {
-      const int j = kb + jj;  // key tile
-      if (!wait_bounded_warp(bar(L::kSFull + t), jj & 1, limit_ns, abort_flag, err)) {
-        ok = false;
+    for (int k = 0; ok; ++k) {
+      int item;
+      if (!read_item(k, item, err) || item < 0) break;
+      const FwdItem w = fwd_item<kCausal, kSplit>(item, n_kv_all, bh_count, head_group, num_splits);
+      const int qt = t ? w.qt1 : w.qt0;
+      const int n_t = t ? w.n1 : w.n0;
+      const bool active = t == 1 || !w.single;  // this tile stands for a real Q tile
+      float m_run = -INFINITY;  // running (possibly stale) max of scale*log2(e)*s
+      float l_run = 0.f;        // running sum of 2^(x - m_run)
+      if (!dbg_check(tmem_range_ok(s_addr, tmem, 128, L::kTmemCols) &&
+                         tmem_range_ok(o_addr, tmem, D, L::kTmemCols) && qt < n_kv_all &&
+                         w.bh < bh_count && w.split < num_splits,
+                     err, abort_flag))
         break;
-      }
-      tc_fence_after();
-      uint32_t u[128];  // raw fp32 scores of this row
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld_32x32b_x32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
-      tmem_wait_ld();
-      // mask: causal diagonal tile (key > query) and keys past the end.  A
-      // masked score becomes the value that scales to -inf.
-      int lim = L::kBN;
-      if (kCausal && j == qt) lim = r + 1;
-      const int rem = n - j * L::kBN;
-      if (rem < lim) lim = rem;
-      if (lim < L::kBN) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) u[c] = (c < lim) ? u[c] : masked_bits;
-      }
-      // row max of scale*log2(e)*s: the max of s, or its min for a negative scale
-      float mx0 = __uint_as_float(u[0]), mx1 = __uint_as_float(u[1]);
-      float mx2 = __uint_as_float(u[2]), mx3 = __uint_as_float(u[3]);
-      if (neg_scale) {
-#pragma unroll
-        for (int c = 4; c < 128; c += 8) {
-          mx0 = fmin3(mx0, __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
-          mx1 = fmin3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
-          mx2 = fmin3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
-          mx3 = fmin3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
+      for (int jj = 0; jj < n_t; ++jj) {
+        const int j = w.kb + jj;  // key tile
+        if (!wait_bounded_warp(bar(L::kSFull + t), s_cnt & 1, limit_ns, abort_flag, err)) {
+          ok = false;
+          break;
         }
-        mx0 = fminf(fmin3(mx0, mx1, mx2), mx3);
-      } else {
-#pragma unroll
-        for (int c = 4; c < 128; c += 8) {
-          mx0 = fmax3(mx0, __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
-          mx1 = fmax3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
-          mx2 = fmax3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
-          mx3 = fmax3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
-        }
-        mx0 = fmaxf(fmax3(mx0, mx1, mx2), mx3);
-      }
-      const float m_tile = mx0 * scale_log2;
-      const bool move = m_tile > m_run + L::kRescaleThreshold;
-      const float alpha = move ? ex2_approx(m_run - m_tile) : 1.0f;
-      if (move) m_run = m_tile;
-      const float neg_m = -m_run;
-      float sum0 = 0.f, sum1 = 0.f;
-      // warp-uniform branch: both paths end in tcgen05.st, which every lane of
-      // the warp must execute together (a lane with lim == 128 masks nothing)
-      if (__any_sync(0xffffffffu, lim < L::kBN)) {
-        // masked tile: a masked key's probability is exactly 0 (also for a
-        // zero scale, where the -inf * 0 product would not be -inf)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int c = q * 32 + e;
-            float p0 = ex2_approx(fmaf(__uint_as_float(u[c]), scale_log2, neg_m));
-            float p1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), scale_log2, neg_m));
-            p0 = (c < lim) ? p0 : 0.f;
-            p1 = (c + 1 < lim) ? p1 : 0.f;
-            sum0 += p0;
-            sum1 += p1;
-            pk[e >> 1] = pack_bf16x2(p0, p1);
-          }
-          tmem_st_32x32b_x16(s_addr + q * 16, pk);
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {  // 32 keys -> 16 packed bf16 pairs -> TMEM
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float a0 = fmaf(__uint_as_float(u[q * 32 + e]), scale_log2, neg_m);
-            const float a1 = fmaf(__uint_as_float(u[q * 32 + e + 1]), scale_log2, neg_m);
-            const float p0 = ex2_approx(a0);
-            const float p1 = ex2_approx(a1);
-            sum0 += p0;
-            sum1 += p1;
-            pk[e >> 1] = pack_bf16x2(p0, p1);
-          }
-          tmem_st_32x32b_x16(s_addr + q * 16, pk);
-        }
-      }
-      l_run = l_run * alpha + (sum0 + sum1);
-      if (jj > 0 && __any_sync(0xffffffffu, move)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld_32x32b_x32(o_addr + c * 32, u);
+        ++s_cnt;
+        tc_fence_after();
+        uint32_t u[128];  // raw fp32 scores of this row
+        int lim = L::kBN;
+        if (kCausal && j == qt) lim = r + 1;
+        const int rem = n - j * L::kBN;
+        if (rem < lim) lim = rem;
+        // From the second key tile on (unmasked tiles, positive scale) the
+        // exponentials are taken against the running max right away, while the
+        // tile's max is found alongside, and the second half of the row loads
+        // while the first half is exponentiated: the max is off the critical
+        // path.  A row's probabilities then reach 2^(tile max - running max);
+        // up to 2^20 that is harmless (bf16 P and the fp32 sums have the range,
+        // and O and l stay relative to the same max), so only a jump beyond
+        // that -- never seen with these inputs -- redoes the tile.
+        if (jj > 0 && !neg_scale && !__any_sync(0xffffffffu, lim < L::kBN)) {
+          tmem_ld_32x32b_x32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          tmem_ld_32x32b_x32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
           tmem_wait_ld();
+          regs_ready(*reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          regs_ready(*reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          tmem_ld_32x32b_x32(s_addr + 64, *reinterpret_cast<uint32_t(*)[32]>(&u[64]));
+          tmem_ld_32x32b_x32(s_addr + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
+          const float neg_m0 = -m_run;
+          float mxa = -INFINITY, mxb = -INFINITY;
+          float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st_32x32b_x32(o_addr + c * 32, u);
+          for (int q = 0; q < 4; ++q) {
+            if (q == 2) {
+              tmem_wait_ld();
+              regs_ready(*reinterpret_cast<uint32_t(*)[32]>(&u[64]));
+              regs_ready(*reinterpret_cast<uint32_t(*)[32]>(&u[96]));
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float s0 = __uint_as_float(u[q * 32 + e]), s1 = __uint_as_float(u[q * 32 + e + 1]);
+              if (e & 2) mxb = fmax3(mxb, s0, s1); else mxa = fmax3(mxa, s0, s1);
+              const float p0 = ex2_approx(fmaf(s0, scale_log2, neg_m0));
+              const float p1 = ex2_approx(fmaf(s1, scale_log2, neg_m0));
+              sum0 += p0;
+              sum1 += p1;
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
+            tmem_st_32x32b_x16(s_addr + q * 16, pk);
+          }
+          const float m_tile = fmaxf(mxa, mxb) * scale_log2;
+          const bool move = m_tile > m_run + L::kSpecRedoThreshold;
+          float alpha = 1.0f;
+          if (__any_sync(0xffffffffu, move)) {  // redo the tile against the new max
+            alpha = move ? ex2_approx(m_run - m_tile) : 1.0f;
+            if (move) m_run = m_tile;
+            const float neg_m = -m_run;
+            sum0 = 0.f;
+            sum1 = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(u[q * 32 + e]), scale_log2, neg_m));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(u[q * 32 + e + 1]), scale_log2, neg_m));
+                sum0 += p0;
+                sum1 += p1;
+                pk[e >> 1] = pack_bf16x2(p0, p1);
+              }
+              tmem_st_32x32b_x16(s_addr + q * 16, pk);
+            }
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t v[32];
+              tmem_ld_32x32b_x32(o_addr + c * 32, v);
+              tmem_wait_ld_regs(v);
+#pragma unroll
+              for (int i2 = 0; i2 < 32; ++i2) v[i2] = __float_as_uint(__uint_as_float(v[i2]) * alpha);
+              tmem_st_32x32b_x32(o_addr + c * 32, v);
+            }
+          }
+          l_run = l_run * alpha + (sum0 + sum1);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(L::kPFull + t));
+          continue;
         }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::kPFull + t));
-    }
-
-    // ------------------------------------------------------------ epilogue
-    if (kSplit) {
-      // partial result of this split (rows of a Q tile past the last tile of
-      // the sequence do not exist in the partial buffers)
-      if (n_t > 0 && ok)
-        ok = wait_bounded_warp(bar(L::kOFinal + t), 0, limit_ns, abort_flag,
-                               err_fwd | kErrRoleEpilogue);
-      if (ok && qt < n_kv_all) {
-        const size_t tile_idx = (static_cast<size_t>(blockIdx.z) * gridDim.x + bh) * n_kv_all + qt;
-        float* po = part_o + tile_idx * 128 * D + r * 4;
-        if (n_t > 0) {
-          tc_fence_after();
-          const float inv_l = 1.0f / l_run;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld_32x32b_x32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
+        tmem_wait_ld_regs(u);
+        // mask: causal diagonal tile (key > query) and keys past the end.  A
+        // masked score becomes the value that scales to -inf.
+        if (lim < L::kBN) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) u[c] = (c < lim) ? u[c] : masked_bits;
+        }
+        // row max of scale*log2(e)*s: the max of s, or its min for a negative scale
+        float mx0 = __uint_as_float(u[0]), mx1 = __uint_as_float(u[1]);
+        float mx2 = __uint_as_float(u[2]), mx3 = __uint_as_float(u[3]);
+        if (neg_scale) {
+#pragma unroll
+          for (int c = 4; c < 128; c += 8) {
+            mx0 = fmin3(mx0, __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
+            mx1 = fmin3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
+            mx2 = fmin3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
+            mx3 = fmin3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
+          }
+          mx0 = fminf(fmin3(mx0, mx1, mx2), mx3);
+        } else {
+#pragma unroll
+          for (int c = 4; c < 128; c += 8) {
+            mx0 = fmax3(mx0, __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
+            mx1 = fmax3(mx1, __uint_as_float(u[c + 2]), __uint_as_float(u[c + 3]));
+            mx2 = fmax3(mx2, __uint_as_float(u[c + 4]), __uint_as_float(u[c + 5]));
+            mx3 = fmax3(mx3, __uint_as_float(u[c + 6]), __uint_as_float(u[c + 7]));
+          }
+          mx0 = fmaxf(fmax3(mx0, mx1, mx2), mx3);
+        }
+        const float m_tile = mx0 * scale_log2;
+        const bool move = m_tile > m_run + L::kRescaleThreshold;
+        const float alpha = move ? ex2_approx(m_run - m_tile) : 1.0f;
+        if (move) m_run = m_tile;
+        const float neg_m = -m_run;
+        float sum0 = 0.f, sum1 = 0.f;
+        // warp-uniform branch: both paths end in tcgen05.st, which every lane of
+        // the warp must execute together (a lane with lim == 128 masks nothing)
+        if (__any_sync(0xffffffffu, lim < L::kBN)) {
+          // masked tile: a masked key's probability is exactly 0 (also for a
+          // zero scale, where the -inf * 0 product would not be -inf)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int c = q * 32 + e;
+              float p0 = ex2_approx(fmaf(__uint_as_float(u[c]), scale_log2, neg_m));
+              float p1 = ex2_approx(fmaf(__uint_as_float(u[c + 1]), scale_log2, neg_m));
+              p0 = (c < lim) ? p0 : 0.f;
+              p1 = (c + 1 < lim) ? p1 : 0.f;
+              sum0 += p0;
+              sum1 += p1;
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
+            tmem_st_32x32b_x16(s_addr + q * 16, pk);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {  // 32 keys -> 16 packed bf16 pairs -> TMEM
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float a0 = fmaf(__uint_as_float(u[q * 32 + e]), scale_log2, neg_m);
+              const float a1 = fmaf(__uint_as_float(u[q * 32 + e + 1]), scale_log2, neg_m);
+              const float p0 = ex2_approx(a0);
+              const float p1 = ex2_approx(a1);
+              sum0 += p0;
+              sum1 += p1;
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
+            tmem_st_32x32b_x16(s_addr + q * 16, pk);
+          }
+        }
+        l_run = l_run * alpha + (sum0 + sum1);
+        if (jj > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t u[32];
             tmem_ld_32x32b_x32(o_addr + c * 32, u);
-            tmem_wait_ld();
+            tmem_wait_ld_regs(u);
 #pragma unroll
-            for (int g = 0; g < 8; ++g)
-              *reinterpret_cast<float4*>(po + (c * 8 + g) * 512) =
-                  make_float4(__uint_as_float(u[4 * g]) * inv_l, __uint_as_float(u[4 * g + 1]) * inv_l,
-                              __uint_as_float(u[4 * g + 2]) * inv_l,
-                              __uint_as_float(u[4 * g + 3]) * inv_l);
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+            tmem_st_32x32b_x32(o_addr + c * 32, u);
           }
-        } else {
-#pragma unroll
-          for (int g = 0; g < D / 4; ++g)
-            *reinterpret_cast<float4*>(po + g * 512) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        part_lse[tile_idx * 128 + r] = (n_t > 0) ? m_run + __log2f(l_run) : -INFINITY;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::kPFull + t));
       }
-    } else {
-      if (ok) ok = wait_bounded_warp(bar(L::kOFinal + t), 0, limit_ns, abort_flag,
-                                err_fwd | kErrRoleEpilogue);
-      const uint32_t stage = sb + (t ? L::kOffQ1 : L::kOffQ0);  // Q_t is dead: stage O_t there
-      if (ok) {
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      // the final O_t is complete once the tile's last P V is; it is read out
+      // of TMEM before this warp group arrives on the next item's P, which is
+      // what the next item's first P V (overwriting O_t) waits for
+      if (n_t > 0) {
+        if (!wait_bounded_warp(bar(L::kOFinal + t), of_cnt & 1, limit_ns, abort_flag,
+                               err_fwd | kErrRoleEpilogue)) {
+          ok = false;
+          break;
+        }
+        ++of_cnt;
         tc_fence_after();
+      }
+      if (kSplit) {
+        // partial result of this split for a real Q tile
+        if (active) {
+          const size_t tile_idx =
+              (static_cast<size_t>(w.split) * bh_count + w.bh) * n_kv_all + qt;
+          if (!dbg_check(tile_idx < static_cast<size_t>(num_splits) * bh_count * n_kv_all, err,
+                         abort_flag))
+            break;
+          float* po = part_o + tile_idx * 128 * D + r * 4;
+          if (n_t > 0) {
+            const float inv_l = 1.0f / l_run;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t u[32];
+              tmem_ld_32x32b_x32(o_addr + c * 32, u);
+              tmem_wait_ld_regs(u);
+#pragma unroll
+              for (int g = 0; g < 8; ++g)
+                *reinterpret_cast<float4*>(po + (c * 8 + g) * 512) = make_float4(
+                    __uint_as_float(u[4 * g]) * inv_l, __uint_as_float(u[4 * g + 1]) * inv_l,
+                    __uint_as_float(u[4 * g + 2]) * inv_l, __uint_as_float(u[4 * g + 3]) * inv_l);
+            }
+          } else {
+#pragma unroll
+            for (int g = 0; g < D / 4; ++g)
+              *reinterpret_cast<float4*>(po + g * 512) = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          part_lse[tile_idx * 128 + r] = (n_t > 0) ? m_run + __log2f(l_run) : -INFINITY;
+        }
+      } else if (active) {
+        // O_t / l as bf16, each thread storing its own row (rows >= N are not
+        // written); the L2 merges the 16-byte pieces of a row into full lines
         const float inv_l = 1.0f / l_run;
-        const uint32_t orow = stage + r * 128;
+        const int row = qt * L::kBM + r;
+        __nv_bfloat16* orow = o_out + (static_cast<size_t>(w.bh) * n + row) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t u[32];
           tmem_ld_32x32b_x32(o_addr + c * 32, u);
-          tmem_wait_ld();
+          tmem_wait_ld_regs(u);
+          if (row < n) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int jj = c * 4 + q;  // 16-byte chunk index within the row
-            const uint32_t addr = orow + (jj >> 3) * 16384 + ((((jj & 7) ^ (r & 7))) << 4);
-            st_shared_v4(addr,
-                         pack_bf16x2(__uint_as_float(u[8 * q + 0]) * inv_l,
-                                     __uint_as_float(u[8 * q + 1]) * inv_l),
-                         pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv_l,
-                                     __uint_as_float(u[8 * q + 3]) * inv_l),
-                         pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv_l,
-                                     __uint_as_float(u[8 * q + 5]) * inv_l),
-                         pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv_l,
-                                     __uint_as_float(u[8 * q + 7]) * inv_l));
+            for (int q = 0; q < 4; ++q)
+              st_global_v4(orow + c * 32 + q * 8,
+                           pack_bf16x2(__uint_as_float(u[8 * q + 0]) * inv_l,
+                                       __uint_as_float(u[8 * q + 1]) * inv_l),
+                           pack_bf16x2(__uint_as_float(u[8 * q + 2]) * inv_l,
+                                       __uint_as_float(u[8 * q + 3]) * inv_l),
+                           pack_bf16x2(__uint_as_float(u[8 * q + 4]) * inv_l,
+                                       __uint_as_float(u[8 * q + 5]) * inv_l),
+                           pack_bf16x2(__uint_as_float(u[8 * q + 6]) * inv_l,
+                                       __uint_as_float(u[8 * q + 7]) * inv_l));
           }
         }
-        const int row = qt * L::kBM + r;
         if (row < n)
-          lse_out[static_cast<size_t>(bh) * n + row] =
+          lse_out[static_cast<size_t>(w.bh) * n + row] =
               (m_run + __log2f(l_run)) * 0.69314718055994530942f;
-        fence_proxy_async_smem();
-      }
-      tc_fence_before();
-      named_barrier_sync(1 + t, 128);  // every warp of this tile reaches this, ok or not
-      if (r == 0 && ok && !*abort_flag && qt * L::kBM < n) {
-        for (int db = 0; db < kDBlk; ++db)
-          tma_store_3d(&tm_o, stage + db * 16384, db * 64, qt * L::kBM, bh);
-        bulk_commit_group();
-        bulk_wait_group_0();
       }
     }
   }
@@ -467,6 +704,7 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
   }
+  if (threadIdx.x == 0) sched_finish(sched_slot);
 }
 
 // Merge of the split partial results, page "FlashAttention 为什么能节省显存并提速,

@@ -118,7 +118,8 @@ __global__ void __launch_bounds__(256, 1)
       bool ok = true;
       for (int j = 0; ok && j < nt; ++j) {
         const int kv = j & 1;
-        if (!wait_bounded(bar(L::kKvEmpty + kv), ((j >> 1) & 1) ^ 1, limit_ns, abort_flag, err))
+        if (!dbg_check(j * 128 < n, err, abort_flag) ||
+            !wait_bounded(bar(L::kKvEmpty + kv), ((j >> 1) & 1) ^ 1, limit_ns, abort_flag, err))
           break;
         mbar_arrive_expect_tx(bar(L::kKvFull + kv), 2 * L::kTile);
         for (int db = 0; db < kDBlk; ++db) {
@@ -130,7 +131,8 @@ __global__ void __launch_bounds__(256, 1)
         ++nkv;
         for (int i = kv_outer_first_i(kCausal, j); i < nt; ++i, ++q) {
           const int st = q & 1;
-          if (!wait_bounded(bar(L::kQEmpty + st), ((q >> 1) & 1) ^ 1, limit_ns, abort_flag, err)) {
+          if (!dbg_check(i * 128 < n, err, abort_flag) ||
+              !wait_bounded(bar(L::kQEmpty + st), ((q >> 1) & 1) ^ 1, limit_ns, abort_flag, err)) {
             ok = false;
             break;
           }
@@ -242,7 +244,7 @@ __global__ void __launch_bounds__(256, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
         tmem_ld_32x32b_x32(pv + c * 32, u);
-        tmem_wait_ld();
+        tmem_wait_ld_regs(u);
         float o[32];
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
@@ -286,7 +288,7 @@ __global__ void __launch_bounds__(256, 1)
             for (int db = 0; db < kDBlk; ++db)
               tma_store_3d(&tm_o, sb + L::kOffStage + db * 16384, db * 64, pi * 128, bh);
             bulk_commit_group();
-            bulk_wait_group_0();  // the store has read the staging tile
+            bulk_wait_group_read_0();  // the store has read the staging tile
             mbar_arrive(bar(L::kStageFree));
           }
           __syncwarp();
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           tmem_ld_32x32b_x32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
-        tmem_wait_ld();
+        tmem_wait_ld_regs(u);
         int lim = 128;  // keys of this tile the row sees
         if (kCausal && j == i) lim = r + 1;
         const int rem = n - j * 128;

@@ -115,6 +115,13 @@ __device__ __forceinline__ void bulk_wait_group_0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Waits until every committed bulk store has finished READING its shared
+// memory source (the global writes may still be in flight; they are visible
+// once the kernel completes).  Enough before reusing or releasing the source.
+__device__ __forceinline__ void bulk_wait_group_read_0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -181,6 +188,27 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// tcgen05.ld fills its destination registers asynchronously: they hold the
+// loaded values only after tcgen05.wait::ld.  To the compiler, though, the
+// load's asm statement defines them at once and the wait shares no register
+// with them, so arithmetic on the values could be scheduled above the wait
+// (one build computed a row minimum from not-yet-loaded registers that way).
+// After the wait, the registers pass through this empty volatile statement,
+// which keeps its place after the wait (volatile statements are not
+// reordered) and redefines them, so every use comes after it.
+__device__ __forceinline__ void regs_ready(uint32_t (&r)[32]) {
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
+
+// tcgen05.wait::ld, then every register of r (a multiple of 32) marked ready.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[N]) {
+  static_assert(N % 32 == 0, "whole 32-register chunks");
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < N; i += 32) regs_ready(*reinterpret_cast<uint32_t(*)[32]>(&r[i]));
 }
 
 __device__ __forceinline__ void tmem_wait_st() {
@@ -282,10 +310,12 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// Two two-input minimums: the three-input min.f32 form, written like fmax3
+// above, gave all-NaN rows in the forward's negative-scale path when the
+// softmax warps ran under setmaxnreg (the same code without the register
+// split, or with this form, is exact).  That path is not the hot one.
 __device__ __forceinline__ float fmin3(float a, float b, float c) {
-  float r;
-  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
+  return fminf(fminf(a, b), c);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -310,6 +340,15 @@ __device__ __forceinline__ void st_global_v4(void* addr, uint32_t a, uint32_t b,
 
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {

@@ -16,7 +16,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
+# FA_LIBRARY selects another build of the same library (e.g. the bounds-checked
+# libfa_b200_debug.so); by default the release build next to this file.
+LIB_PATH = os.environ.get("FA_LIBRARY") or os.path.join(_HERE, "libfa_b200.so")
 
 FA_OK = 0
 STATUS_NAMES = {

@@ -28,11 +28,19 @@
  * Causal masking keeps key j for query i iff j <= i.
  *
  * Ownership: the caller owns every buffer (device memory) and the stream.  The
- * library allocates no device memory, keeps no per-call state, and never
- * synchronises except inside fa_check_device_error and fa_timing_end.  Calls
- * are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ * library allocates no device memory at call time and never synchronises
+ * except inside fa_check_device_error and fa_timing_end.  Calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  * stream).  Concurrent calls on different streams must use distinct output
  * and workspace buffers.
+ *
+ * Library-owned device state (static device arrays, part of the loaded
+ * library, never allocated per call): the error word; the work counters of
+ * the persistent kernels (16384 slots of 16 bytes: each launch takes the next
+ * slot of a per-device sequence, the first CTA to ask for work in a launch
+ * starts the slot's count afresh and the last CTA to finish clears it, so
+ * concurrent launches and replays of a captured CUDA graph each count their
+ * own work); and the scratch of fa_bwd_noalloc.
  *
  * Errors: arguments are checked before anything is launched; a failing check
  * returns its code and launches nothing.  A launch failure returns
@@ -76,7 +84,10 @@ typedef enum {
  *             exp(scale * q_i . k_j) over unmasked keys j).
  *   causal  : 0 = every key, nonzero = keys j <= i only.
  *   scale   : any finite float (the usual value is 1/sqrt(d)).
- * Deterministic: the same inputs give bitwise the same outputs.
+ * Deterministic: the same inputs give bitwise the same outputs (each pair of
+ * 128-row Q tiles is computed by one CTA in a fixed order, whichever CTA it
+ * lands on).  One persistent CTA per SM takes the (head, Q-tile pair) work
+ * items longest first from a per-launch counter.
  */
 FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                  int B, int H, int N, int d, int causal, float scale, void* stream);

@@ -29,7 +29,7 @@ def _run_and_check(q, k, v, causal, scale, slices=None):
 
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("n", [1, 2, 127, 128, 129, 300, 1000])
+@pytest.mark.parametrize("n", [1, 2, 127, 128, 129, 300, 384, 640, 1000])
 def test_fwd_small_shapes(d, causal, n):
     w = Workload("small", 1, 2, n, d, seed_base=17 + n)
     x = make_inputs(w, DEV, with_do=False)
@@ -146,3 +146,53 @@ def test_fwd_any_finite_scale(scale, causal):
     w = Workload("scale", 1, 2, 300, 128, seed_base=13)
     x = make_inputs(w, DEV, with_do=False)
     _run_and_check(x["q"], x["k"], x["v"], causal, scale)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_many_heads_in_groups(causal):
+    """More than 48 heads run in launch groups of 32 with a partial last group
+    (B*H = 50): the heads at both ends of each group are right;
+    N = 700 (6 Q tiles) and N = 520 (5 Q tiles, so the last pair has a single
+    tile) run inside groups."""
+    for n in (700, 520):
+        w = Workload("groups", 2, 25, n, 64, seed_base=19 + n)
+        x = make_inputs(w, DEV, with_do=False)
+        heads = [0, 1, 31, 32, 33, 48, 49]
+        _run_and_check(x["q"], x["k"], x["v"], causal, w.scale,
+                       slices=[(i // 25, i % 25) for i in heads])
+
+
+def test_fwd_graph_replay_and_concurrent_streams():
+    """The persistent forward hands out work from a per-launch counter: a
+    captured launch replayed several times, and launches running at the same
+    time on several streams, all give the eager single-stream result bit for
+    bit (the forward is deterministic)."""
+    w = Workload("graph", 2, 8, 1000, 128, seed_base=23)
+    x = make_inputs(w, DEV, with_do=False)
+    ref_o, ref_lse = fa.forward(x["q"], x["k"], x["v"], causal=True)
+    fa.check_device_error()
+    o = torch.empty_like(ref_o)
+    lse = torch.empty_like(ref_lse)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=side):
+        fa.forward(x["q"], x["k"], x["v"], causal=True, out=o, lse=lse)
+    for _ in range(3):
+        o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, ref_o) and torch.equal(lse, ref_lse)
+    del g
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    outs = [(torch.empty_like(ref_o), torch.empty_like(ref_lse)) for _ in streams]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for s, (oo, ll) in zip(streams, outs):
+            with torch.cuda.stream(s):
+                oo.fill_(float("nan"))
+                fa.forward(x["q"], x["k"], x["v"], causal=True, out=oo, lse=ll)
+    torch.cuda.synchronize()
+    fa.check_device_error()
+    for oo, ll in outs:
+        assert torch.equal(oo, ref_o) and torch.equal(ll, ref_lse)
