@@ -170,25 +170,14 @@ def test_clock_sampler_decodes_nvml_reasons():
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
     import bench
 
-    class FakeNvml:  # read-only queries of a GPU at 1800 of 1965 MHz under the power cap
-        NVML_CLOCK_SM = 1
-
-        @staticmethod
-        def nvmlDeviceGetClockInfo(h, kind):
-            return 1800
-
-        @staticmethod
-        def nvmlDeviceGetMaxClockInfo(h, kind):
-            return 1965
-
-        @staticmethod
-        def nvmlDeviceGetCurrentClocksEventReasons(h):
-            return 0x4 | 0x1  # sw power cap, plus the (ignored) idle bit
-
-    c = bench.ClockSampler(0)
-    c._nvml, c._handle, c.source = FakeNvml, object(), "nvml"
-    for _ in range(3):
-        c._sample_nvml()
+    # NVML samples (ns, SM MHz, max MHz, reason bits) of a GPU at 1800 of 1965 MHz
+    # under the power cap (0x4) with the ignored idle bit (0x1); the first and
+    # last fall outside the timed region [100, 400].
+    raw = [(50, 1965, 1965, 0x1)] + [(t, 1800, 1965, 0x4 | 0x1) for t in (100, 250, 400)] \
+        + [(450, 1965, 1965, 0x8)]
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.samples, c.source = [], "nvml"
+    c.add_nvml_samples(raw, 100, 400)
     s = c.summary()
     assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
     assert s["reasons"] == ["sw_power_cap"] and s["source"] == "nvml"
@@ -210,3 +199,18 @@ def test_roofline_entry_for_the_dominant_kernel():
     r = bench.roofline_entry({"bwd_pre": 1.0, "fwd": 0.5}, {"bwd_pre": 0.1, "fwd": 0.05},
                              {"fwd": 1e9}, {"hbm_gbs": 6542.4}, "measured", lambda k: None)
     assert r["bound"] == "hbm" and r["frac"] is None
+
+
+def test_clock_sampler_keeps_nearest_sample_for_a_short_region():
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+
+    raw = [(0, 1900, 1965, 0x0), (1000, 1700, 1965, 0x40)]
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.samples, c.source = [], "nvml"
+    c.add_nvml_samples(raw, 700, 800)  # no sample inside: the one at 1000 is nearest
+    s = c.summary()
+    assert s["samples"] == 1 and s["sm_mhz"] == 1700
+    assert s["reasons"] == ["hw_thermal_slowdown"]
