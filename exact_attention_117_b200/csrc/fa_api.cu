@@ -41,21 +41,33 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 tensor [BH, rows, cols] (cols innermost), box = 64 cols x box_rows rows
-// x 1, 128-byte swizzle.  Out-of-range loads read zeros; stores are clipped.
-bool encode_bf16_3d(CUtensorMap* map, const void* ptr, int cols, int rows, int bh, int box_rows) {
+// bf16 tensor [BH, rows, cols] (cols innermost), box = box_cols cols x box_rows
+// rows x 1.  Out-of-range loads read zeros; stores are clipped.
+bool encode_bf16_3d_box(CUtensorMap* map, const void* ptr, int cols, int rows, int bh,
+                        int box_cols, int box_rows, CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(bh)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2,
                            static_cast<cuuint64_t>(cols) * 2 * static_cast<cuuint64_t>(rows)};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// The operand layout of the kernels: 64 cols (128 bytes) x box_rows, 128-byte swizzle.
+bool encode_bf16_3d(CUtensorMap* map, const void* ptr, int cols, int rows, int bh, int box_rows) {
+  return encode_bf16_3d_box(map, ptr, cols, rows, bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// The forward's output: 32 x 32 boxes (64-byte rows), 64-byte swizzle, one per
+// softmax warp and 32 output columns (fa::FwdLayout::kOffStage).
+bool encode_fwd_out(CUtensorMap* map, const void* o, int d, int N, int bh) {
+  return encode_bf16_3d_box(map, o, d, N, bh, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 // --------------------------------------------------------------- timing
@@ -173,7 +185,8 @@ uint32_t next_sched_slot(int dev) {
 
 template <int D, bool C, bool kSplit>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     void* o, float* lse, int BH, int N, float scale_log2, cudaStream_t st,
+                     const CUtensorMap& mo, float* lse, int BH, int N, float scale_log2,
+                     cudaStream_t st,
                      int num_splits = 1, float* part_o = nullptr, float* part_lse = nullptr) {
   using L = fa::FwdLayout<D>;
   static bool attr_set[kMaxDevices] = {};
@@ -194,10 +207,14 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   const int n_items = static_cast<int>(items);
   const int grid = std::min(n_items, sm_count(dev));  // persistent: one CTA per SM
   const uint32_t slot = next_sched_slot(dev);
+  // the kernel's masked score (-inf after scaling) needs a nonzero factor; at
+  // 1e-30 every scaled score of a finite input is 0 to fp32 accuracy, as it is
+  // for a zero scale
+  if (std::fabs(scale_log2) < 1e-30f) scale_log2 = std::signbit(scale_log2) ? -1e-30f : 1e-30f;
   {
     LaunchTimer timer(st, FA_KERNEL_FWD);
     fa::fwd_kernel<D, C, kSplit><<<grid, 384, L::kSmemAlloc, st>>>(
-        mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse, N, BH, scale_log2, kWaitLimitNs,
+        mq, mk, mv, mo, lse, N, BH, scale_log2, kWaitLimitNs,
         num_splits, part_o, part_lse, head_group, n_items, slot);
   }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -351,17 +368,17 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_ALIGN;
   const int bh = B * H;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
-      !encode_bf16_3d(&mv, v, d, N, bh, 128))
+      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_fwd_out(&mo, o, d, N, bh))
     return FA_ERR_CUDA;
   const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
-    return causal ? launch_fwd<64, true, false>(mq, mk, mv, o, lse, bh, N, scale_log2, s)
-                  : launch_fwd<64, false, false>(mq, mk, mv, o, lse, bh, N, scale_log2, s);
-  return causal ? launch_fwd<128, true, false>(mq, mk, mv, o, lse, bh, N, scale_log2, s)
-                : launch_fwd<128, false, false>(mq, mk, mv, o, lse, bh, N, scale_log2, s);
+    return causal ? launch_fwd<64, true, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
+                  : launch_fwd<64, false, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
+  return causal ? launch_fwd<128, true, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s)
+                : launch_fwd<128, false, false>(mq, mk, mv, mo, lse, bh, N, scale_log2, s);
 }
 
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits) {
@@ -396,14 +413,14 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   fa_status r;
   if (d == 64)
-    r = causal ? launch_fwd<64, true, true>(mq, mk, mv, nullptr, lse, bh, N, scale_log2, s,
+    r = causal ? launch_fwd<64, true, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
                                             num_splits, part_o, part_lse)
-               : launch_fwd<64, false, true>(mq, mk, mv, nullptr, lse, bh, N, scale_log2, s,
+               : launch_fwd<64, false, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
                                              num_splits, part_o, part_lse);
   else
-    r = causal ? launch_fwd<128, true, true>(mq, mk, mv, nullptr, lse, bh, N, scale_log2, s,
+    r = causal ? launch_fwd<128, true, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
                                              num_splits, part_o, part_lse)
-               : launch_fwd<128, false, true>(mq, mk, mv, nullptr, lse, bh, N, scale_log2, s,
+               : launch_fwd<128, false, true>(mq, mk, mv, mq, lse, bh, N, scale_log2, s,
                                               num_splits, part_o, part_lse);
   if (r != FA_OK) return r;
   {
