@@ -33,7 +33,14 @@
 // products are read out of TMEM by a separate warp group and added into the
 // fp32 accumulator with vector atomic adds.  The accumulator keeps each
 // 128-row tile as [D/4 column groups][128 rows][4 floats] so that those adds
-// are coalesced.
+// are coalesced.  For d = 128 the 64 KB of adds of one Q tile are paced, an
+// 80 ns sleep after each pair of vector adds (about 1.3 us in all, under half
+// of a Q-loop iteration): issued as one burst they queue ahead of the next
+// tile loads and stretch every iteration (B200: 857 -> 940 TFLOP/s for this
+// kernel at B=2 H=16 N=4096, 880-930 -> 988 at B=1 H=32 N=16384).  Sleeping
+// for most of the iteration instead (2.4 us) makes the read-out fall behind,
+// and dP of the tile after next waits for it: 650 TFLOP/s.  For d = 64 pacing
+// measured slightly slower.
 //
 // Warp roles (384 threads): warp 0 TMA producer; warp 1 TMEM allocator and MMA
 // issuer; warp 2 builds the LSE / D slabs; warps 4-7 compute P^T / dS^T
@@ -120,6 +127,8 @@ __device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
 // kDq = false (deterministic backward): no dQ MMA and no atomics here; dQ
 // comes from dq_pass_kernel.  dP_{i+1} then only waits for dS_i to be formed.
 constexpr int kHeadGroup = 8;
+// pause after each pair of dQ vector adds (d = 128)
+constexpr uint32_t kAddGapNs = 80;
 
 template <int D, bool kCausal, bool kDq>
 __global__ void __launch_bounds__(384, 1)
@@ -562,9 +571,11 @@ __global__ void __launch_bounds__(384, 1)
       float* dst = dq_acc + (static_cast<size_t>(bh) * n_q + static_cast<size_t>(i)) * 128 * D +
                    static_cast<size_t>(c) * 4;
 #pragma unroll
-      for (int q = 0; q < D / 4; ++q)
+      for (int q = 0; q < D / 4; ++q) {
         red_add_v4(dst + q * 512, __uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
                    __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
+        if (D == 128 && (q & 1)) __nanosleep(kAddGapNs);
+      }
     }
   }
 

@@ -39,6 +39,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// May suspend the thread for a while (a hardware-chosen limit) before giving
+// up; the bounded waits of common.cuh loop on it.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
