@@ -57,6 +57,10 @@ def rank_workload(w, rank):
     return dataclasses.replace(w, seed_base=w.seed_base + 1000 * rank)
 
 
+# groups of (b, h) slices in the end-to-end leg (copies overlap compute)
+E2E_CHUNKS = 4
+
+
 def max_over_ranks(values, world, device=None):
     """Element-wise max of a list of floats over all ranks (max-over-ranks timing)."""
     import torch
@@ -454,33 +458,81 @@ def run_ours(args, w, rank, world, local_rank):
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
 
+        # The (b, h) slices are independent problems, so the step runs as E2E_CHUNKS
+        # groups of slices (each a [1, slices, N, d] call) on three streams:
+        # inputs of group c+1 copy in while group c computes and group c-1's
+        # results copy out (the two copy directions use separate engines).  A
+        # group's buffers are reused only after the previous step is done with
+        # them: its copy-in waits for that step's compute of the group, its
+        # compute for that step's copy-out.
+        bh = w.B * w.H
+        n_chunks = max(1, min(E2E_CHUNKS, bh))
+        bounds = [(c * bh // n_chunks, (c + 1) * bh // n_chunks) for c in range(n_chunks)]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        s_comp = stream
+
+        def flat(t):  # [1, B*H, ...] view of a [B, H, ...] tensor
+            return t.view(1, bh, *t.shape[2:])
+
+        ev_comp = [None] * n_chunks  # last compute of each group
+        ev_out = [None] * n_chunks   # last copy-out of each group
+
         def e2e_step():
-            for n in dev_in:
-                dev_in[n].copy_(host[n], non_blocking=True)
-            fa.forward(dev_in["q"], dev_in["k"], dev_in["v"], causal=causal, scale=w.scale,
-                       out=o, lse=lse, stream=stream)
-            fa.backward(dev_in["q"], dev_in["k"], dev_in["v"], o, lse, dev_in["do"],
-                        causal=causal, scale=w.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
-                        stream=stream)
-            for n, src in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
-                outs_host[n].copy_(src, non_blocking=True)
+            for c, (a, b) in enumerate(bounds):
+                with torch.cuda.stream(s_in):
+                    if ev_comp[c] is not None:
+                        s_in.wait_event(ev_comp[c])
+                    for n in dev_in:
+                        flat(dev_in[n])[:, a:b].copy_(flat(host[n])[:, a:b], non_blocking=True)
+                    ev_i = torch.cuda.Event()
+                    ev_i.record(s_in)
+                s_comp.wait_event(ev_i)
+                if ev_out[c] is not None:
+                    s_comp.wait_event(ev_out[c])
+                qc, kc, vc, doc = (flat(dev_in[n])[:, a:b] for n in ("q", "k", "v", "do"))
+                oc, lc = flat(o)[:, a:b], flat(lse)[:, a:b]
+                fa.forward(qc, kc, vc, causal=causal, scale=w.scale, out=oc, lse=lc,
+                           stream=s_comp)
+                fa.backward(qc, kc, vc, oc, lc, doc, causal=causal, scale=w.scale,
+                            dq=flat(dq)[:, a:b], dk=flat(dk)[:, a:b], dv=flat(dv)[:, a:b],
+                            workspace=ws, stream=s_comp)
+                ev_c = torch.cuda.Event()
+                ev_c.record(s_comp)
+                ev_comp[c] = ev_c
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_c)
+                    for n, src in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+                        flat(outs_host[n])[:, a:b].copy_(flat(src)[:, a:b], non_blocking=True)
+                    ev_o = torch.cuda.Event()
+                    ev_o.record(s_out)
+                    ev_out[c] = ev_o
+
+        def join():  # the timing stream waits for every copy-out issued so far
+            for ev in ev_out:
+                if ev is not None:
+                    stream.wait_event(ev)
 
         for _ in range(2):
             e2e_step()
+        join()
         barrier()
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
         for _ in range(args.steps):
             e2e_step()
+        join()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         e2e_ms = max_over_ranks([e0.elapsed_time(e1)], world, dev)[0] / args.steps
         e2e = {"value": job_tflops(fwd_f + bwd_f, world, e2e_ms), "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "path": "pinned host -> device copy, fa_fwd + fa_bwd through the C ABI, "
-                       "outputs copied back to pinned host"}
+               "path": f"pinned host -> device copy, fa_fwd + fa_bwd through the C ABI, outputs "
+                       f"copied back to pinned host; {n_chunks} groups of (b, h) slices "
+                       f"pipelined over copy-in, compute and copy-out streams"}
 
     # ------------------------------------------------------- long-context leg
     long_ctx = None
@@ -721,6 +773,8 @@ def run_sweep(args):
     if args.sweep in ("all", "c5"):
         with category("c5"):
             for w in sweep_workloads():
+                if args.case and w.name != args.case:
+                    continue
                 x = make_inputs(w, dev)
                 o = torch.empty_like(x["q"])
                 lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
@@ -739,6 +793,10 @@ def run_sweep(args):
                         fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal,
                                     dq=g[0], dk=g[1], dv=g[2], workspace=ws, stream=stream)
                     tag = f"{w.name} {'causal' if causal else 'full'}"
+                    if args.once:  # two forwards and one backward, untimed (for ncu)
+                        fwd()
+                        step()
+                        continue
                     ms = _time_device(fwd, flush, stream)
                     emit(f"{tag} fwd", fwd_f / (ms * 1e-3) / 1e12, ms)
                     ms = _time_device(step, flush, stream)
@@ -927,7 +985,9 @@ def main():
     ap.add_argument("--sweep", choices=["all", "c5", "splitkv", "kv_outer", "bwd"], default=None,
                     help="supplementary per-case measurements instead of the headline line")
     ap.add_argument("--once", action="store_true",
-                    help="with --sweep kv_outer or bwd: run the cases once, untimed (for ncu)")
+                    help="with --sweep c5, kv_outer or bwd: run the cases once, untimed (for ncu)")
+    ap.add_argument("--case", default=None,
+                    help="with --sweep c5: only this workload (e.g. c5_d64_n4096)")
     ap.add_argument("--traffic", action="store_true",
                     help="one launch per traffic-model case (run under ncu for DRAM bytes)")
     ap.add_argument("--traffic-report", metavar="NCU_CSV", default=None,
