@@ -89,10 +89,12 @@ struct FwdLayout {
   static constexpr int kKEmpty = kKFull + kStages;
   static constexpr int kVFull = kKEmpty + kStages;
   static constexpr int kVEmpty = kVFull + kStages;
-  static constexpr int kSFull = kVEmpty + kStages;  // [2]
-  static constexpr int kPFull = kSFull + 2;         // [2]
-  static constexpr int kOFinal = kPFull + 2;        // [2]
-  static constexpr int kItemFull = kOFinal + 2;     // [2]
+  // S ready / P ready, one barrier per score buffer (two, or three at d = 64)
+  static constexpr int kSFull = kVEmpty + kStages;  // [3]
+  static constexpr int kPFull = kSFull + 3;         // [3]
+  static constexpr int kOFinal = kPFull + 3;        // [2]
+  static constexpr int kPvDone = kOFinal + 2;       // [2] one phase per P V of the tile
+  static constexpr int kItemFull = kPvDone + 2;     // [2]
   static constexpr int kItemEmpty = kItemFull + 2;  // [2]
   static constexpr int kDrain = kItemEmpty + 2;
   static constexpr int kNumBars = kDrain + 1;
@@ -102,8 +104,11 @@ struct FwdLayout {
   static_assert(kOffItems + 8 <= kOffBar + kBarArea, "barrier area too small");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
+  // d = 128: S0, S1, O0, O1 fill the 512 columns.  d = 64: three score buffers
+  // shared by the two tiles, then O0, O1 (see s_ref below).
+  static constexpr bool kThreeS = (D == 64);
   static constexpr uint32_t kColS0 = 0, kColS1 = 128;
-  static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
+  static constexpr uint32_t kColO0 = kThreeS ? 384 : 256, kColO1 = kColO0 + D;
   static constexpr float kRescaleThreshold = 8.0f;    // base-2 units
   static constexpr float kSpecRedoThreshold = 20.0f;  // base-2 units, speculative tiles
   static constexpr uint32_t kLaunchRegs = 168;      // 65536 / 384, rounded down to 8
@@ -154,6 +159,32 @@ __device__ __forceinline__ FwdItem fwd_item(int item, int n_kv_all, int bh_count
   return w;
 }
 
+// Where the score tile S_t(j) of an item lives (n0 key tiles for Q tile 0):
+// its TMEM column, the index of its S-ready / P-ready barriers and the parity
+// of the phase that stands for it.  With two buffers, tile t always uses
+// buffer t and the phases count tile t's key steps (t_steps of them before
+// this one).  With three (d = 64), the score tiles take the buffers in turn
+// in the order the MMA warp issues them -- S_0(0), S_1(0), then per key step
+// S_0(j+1), S_1(j+1) -- so that a tile's next scores are computed into the
+// third buffer while its softmax still reads the current ones; s_base counts
+// the score tiles of earlier items.  A buffer is reused only after the P V
+// that reads it, so its barriers never run two phases ahead of a waiter.
+struct SRef {
+  uint32_t col;
+  int buf;
+  uint32_t parity;
+};
+template <int D>
+__device__ __forceinline__ SRef s_ref(int t, int j, int n0, int s_base, int t_steps) {
+  using L = FwdLayout<D>;
+  if (!L::kThreeS)
+    return {t ? L::kColS1 : L::kColS0, t, static_cast<uint32_t>(t_steps & 1)};
+  // the issue index of S_t(j) in this item: tile 0 has n0 tiles, tile 1 n1 =
+  // n0 or n0 + 1 (or n1 alone when tile 0 idles, n0 = 0)
+  const int k = s_base + ((t == 0) ? 2 * j : (j < n0 ? 2 * j + 1 : n0 + j));
+  return {static_cast<uint32_t>(k % 3) * 128, k % 3, static_cast<uint32_t>((k / 3) & 1)};
+}
+
 // kSplit: an item covers only the key tiles of its split (a contiguous range
 // of ceil(n_kv / num_splits) tiles) and writes, instead of O and LSE, fp32
 // partial results: O_s = u_s / l_s in the tile layout [D/4 column groups][128
@@ -188,7 +219,7 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < L::kNumBars; ++b) {
       uint32_t cnt = 1;
-      if (b == L::kPFull || b == L::kPFull + 1) cnt = 4;
+      if (b >= L::kPFull && b < L::kPFull + 3) cnt = 4;
       if (b == L::kItemEmpty || b == L::kItemEmpty + 1) cnt = L::kItemReaders;
       mbar_init(bar(b), cnt);
     }
@@ -325,22 +356,26 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t id_o = idesc_bf16_f32(128, D, false, true);
       const uint32_t err = err_fwd | kErrRoleMma;
-      auto issue_s = [&](int t, int gi) {  // S_t = Q_t K^T, K from ring position gi
+      int s_base = 0;  // score tiles issued by earlier items
+      // S_t(j) = Q_t K^T, K from ring position gi
+      auto issue_s = [&](int t, int gi, int j, int n0) {
         const uint32_t qa = sb + (t ? L::kOffQ1 : L::kOffQ0);
         const uint32_t ka = sb + L::kOffK + (gi % S) * L::kTile;
-        const uint32_t d_tmem = tmem + (t ? L::kColS1 : L::kColS0);
+        const SRef sr = s_ref<D>(t, j, n0, s_base, 0);
+        const uint32_t d_tmem = tmem + sr.col;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
           mma_bf16_ss(d_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), id_s,
                       kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(L::kSFull + t));
+        tc_commit(bar(L::kSFull + sr.buf));
       };
-      auto issue_pv = [&](int t, int gi, bool first) {  // O_t (+)= P_t V, P_t from TMEM
+      // O_t (+)= P_t(j) V, P_t(j) from TMEM over S_t(j)
+      auto issue_pv = [&](int t, int gi, bool first, int j, int n0) {
         const uint32_t va = sb + L::kOffV + (gi % S) * L::kTile;
         const uint32_t d_tmem = tmem + (t ? L::kColO1 : L::kColO0);
-        const uint32_t a_tmem = tmem + (t ? L::kColS1 : L::kColS0);
+        const uint32_t a_tmem = tmem + s_ref<D>(t, j, n0, s_base, 0).col;
 #pragma unroll
         for (int kk = 0; kk < L::kBN / 16; ++kk)
           mma_bf16_ts(d_tmem, a_tmem + kk * 8, sw128_desc(va + kk * 2048, 16384, 1024), id_o,
@@ -363,8 +398,8 @@ __global__ void __launch_bounds__(384, 1)
         ++q_cnt;
         if (!ok) break;
         tc_fence_after();
-        if (n0 > 0) issue_s(0, g_kv);
-        issue_s(1, g_kv);
+        if (n0 > 0) issue_s(0, g_kv, 0, n0);
+        issue_s(1, g_kv, 0, n0);
         tc_commit(bar(L::kKEmpty + g_kv % S));
         if (n1 == 1) tc_commit(bar(L::kQEmpty));  // the item's last S reads of Q are issued
         for (int jj = 0; jj < n1; ++jj) {
@@ -374,42 +409,66 @@ __global__ void __launch_bounds__(384, 1)
             ok = false;
             break;
           }
-          if (jj < n0) {
-            if (!wait_bounded_warp(bar(L::kPFull + 0), p0 & 1, limit_ns, abort_flag, err)) {
-              ok = false;
-              break;
-            }
-            ++p0;
-            tc_fence_after();
-            issue_pv(0, gi, jj == 0);
-            if (jj == n0 - 1) tc_commit(bar(L::kOFinal + 0));
-          }
           const bool next = jj + 1 < n1;
           const int s1 = (gi + 1) % S;
-          if (next) {
+          // three buffers: tile 0's next scores go into the free buffer before
+          // its current P V; two buffers: after it, into the same buffer
+          if (L::kThreeS && next) {
             if (!wait_bounded_warp(bar(L::kKFull + s1), ((gi + 1) / S) & 1, limit_ns, abort_flag,
                                    err)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            if (jj + 1 < n0) issue_s(0, gi + 1);
+            if (jj + 1 < n0) issue_s(0, gi + 1, jj + 1, n0);
           }
-          if (!wait_bounded_warp(bar(L::kPFull + 1), p1 & 1, limit_ns, abort_flag, err)) {
+          if (jj < n0) {
+            const SRef pr = s_ref<D>(0, jj, n0, s_base, p0);
+            if (!wait_bounded_warp(bar(L::kPFull + pr.buf), pr.parity, limit_ns, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            ++p0;
+            tc_fence_after();
+            issue_pv(0, gi, jj == 0, jj, n0);
+            tc_commit(bar(L::kPvDone + 0));
+            if (jj == n0 - 1) tc_commit(bar(L::kOFinal + 0));
+          }
+          if (next) {
+            if (!L::kThreeS) {
+              if (!wait_bounded_warp(bar(L::kKFull + s1), ((gi + 1) / S) & 1, limit_ns, abort_flag,
+                                     err)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              if (jj + 1 < n0) issue_s(0, gi + 1, jj + 1, n0);
+            } else {
+              // tile 1's next scores into the buffer tile 0's P V has just
+              // been issued from
+              issue_s(1, gi + 1, jj + 1, n0);
+              tc_commit(bar(L::kKEmpty + s1));
+              if (jj + 2 == n1) tc_commit(bar(L::kQEmpty));  // last S reads of Q issued
+            }
+          }
+          const SRef pr1 = s_ref<D>(1, jj, n0, s_base, p1);
+          if (!wait_bounded_warp(bar(L::kPFull + pr1.buf), pr1.parity, limit_ns, abort_flag, err)) {
             ok = false;
             break;
           }
           ++p1;
           tc_fence_after();
-          issue_pv(1, gi, jj == 0);
+          issue_pv(1, gi, jj == 0, jj, n0);
+          tc_commit(bar(L::kPvDone + 1));
           if (jj == n1 - 1) tc_commit(bar(L::kOFinal + 1));
           tc_commit(bar(L::kVEmpty + s));
-          if (next) {
-            issue_s(1, gi + 1);
+          if (next && !L::kThreeS) {
+            issue_s(1, gi + 1, jj + 1, n0);
             tc_commit(bar(L::kKEmpty + s1));
             if (jj + 2 == n1) tc_commit(bar(L::kQEmpty));  // last S reads of Q issued
           }
         }
+        s_base += n0 + n1;
         g_kv += n1;
       }
       // every MMA issued above must finish before TMEM / smem are released
@@ -423,12 +482,22 @@ __global__ void __launch_bounds__(384, 1)
     const int t = (warp >= 8) ? 1 : 0;         // which Q tile
     const int r = threadIdx.x - 128 - 128 * t;  // row inside the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + (t ? L::kColS1 : L::kColS0);
     const uint32_t o_addr = tmem + lane_off + (t ? L::kColO1 : L::kColO0);
     const uint32_t err = err_fwd | kErrRoleSoftmax;
     const bool neg_scale = scale_log2 < 0.f;
     const uint32_t masked_bits = __float_as_uint(neg_scale ? INFINITY : -INFINITY);
     int s_cnt = 0, of_cnt = 0;  // S tiles and final O of this tile seen so far
+    int s_base = 0;             // score tiles of earlier items
+    // Before a rescale of O_t at key step jj > 0: O_t holds the tiles before
+    // jj once their P V has finished.  With two buffers the S_t(jj) seen ready
+    // was issued after that P V, so it has; with three it was issued before it.
+    auto o_current = [&]() -> bool {
+      if (!L::kThreeS) return true;
+      const bool got =
+          wait_bounded_warp(bar(L::kPvDone + t), (s_cnt - 2) & 1, limit_ns, abort_flag, err);
+      tc_fence_after();
+      return got;
+    };
     int st_cnt = 0;             // O boxes this warp has stored (staging buffer st_cnt & 1)
     const int sw = warp - 4;    // softmax warp 0..7: its staging buffers
     bool ok = true;
@@ -441,19 +510,22 @@ __global__ void __launch_bounds__(384, 1)
       const bool active = t == 1 || !w.single;  // this tile stands for a real Q tile
       float m_run = -INFINITY;  // running (possibly stale) max of scale*log2(e)*s
       float l_run = 0.f;        // running sum of 2^(x - m_run)
-      if (!dbg_check(tmem_range_ok(s_addr, tmem, 128, L::kTmemCols) &&
+      if (!dbg_check(tmem_range_ok(tmem + lane_off + L::kColS0, tmem, L::kThreeS ? 384 : 256,
+                                   L::kTmemCols) &&
                          tmem_range_ok(o_addr, tmem, D, L::kTmemCols) && qt < n_kv_all &&
                          w.bh < bh_count && w.split < num_splits,
                      err, abort_flag))
         break;
       for (int jj = 0; jj < n_t; ++jj) {
         const int j = w.kb + jj;  // key tile
-        if (!wait_bounded_warp(bar(L::kSFull + t), s_cnt & 1, limit_ns, abort_flag, err)) {
+        const SRef sr = s_ref<D>(t, jj, w.n0, s_base, s_cnt);
+        if (!wait_bounded_warp(bar(L::kSFull + sr.buf), sr.parity, limit_ns, abort_flag, err)) {
           ok = false;
           break;
         }
         ++s_cnt;
         tc_fence_after();
+        const uint32_t s_addr = tmem + lane_off + sr.col;
         uint32_t u[128];  // raw fp32 scores of this row
         int lim = L::kBN;
         if (kCausal && j == qt) lim = r + 1;
@@ -520,6 +592,10 @@ __global__ void __launch_bounds__(384, 1)
               }
               tmem_st_32x32b_x16(s_addr + q * 16, pk);
             }
+            if (!o_current()) {
+              ok = false;
+              break;
+            }
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t v[32];
@@ -534,7 +610,7 @@ __global__ void __launch_bounds__(384, 1)
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(L::kPFull + t));
+          if (lane == 0) mbar_arrive(bar(L::kPFull + sr.buf));
           continue;
         }
         // The same for a masked tile (the causal diagonal, keys past N): a
@@ -598,6 +674,10 @@ __global__ void __launch_bounds__(384, 1)
               }
               tmem_st_32x32b_x16(s_addr + q * 16, pk);
             }
+            if (!o_current()) {
+              ok = false;
+              break;
+            }
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t v[32];
@@ -612,7 +692,7 @@ __global__ void __launch_bounds__(384, 1)
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(L::kPFull + t));
+          if (lane == 0) mbar_arrive(bar(L::kPFull + sr.buf));
           continue;
         }
 #pragma unroll
@@ -693,6 +773,10 @@ __global__ void __launch_bounds__(384, 1)
         }
         l_run = l_run * alpha + (sum0 + sum1);
         if (jj > 0 && __any_sync(0xffffffffu, move)) {
+          if (!o_current()) {
+            ok = false;
+            break;
+          }
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t u[32];
@@ -706,9 +790,10 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::kPFull + t));
+        if (lane == 0) mbar_arrive(bar(L::kPFull + sr.buf));
       }
       if (!ok) break;
+      s_base += w.n0 + w.n1;
 
       // ---------------------------------------------------------- epilogue
       // the final O_t is complete once the tile's last P V is; it is read out
