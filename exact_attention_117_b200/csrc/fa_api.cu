@@ -64,9 +64,10 @@ bool encode_bf16_3d(CUtensorMap* map, const void* ptr, int cols, int rows, int b
   return encode_bf16_3d_box(map, ptr, cols, rows, bh, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// The forward's output: 32 x 32 boxes (64-byte rows), 64-byte swizzle, one per
-// softmax warp and 32 output columns (fa::FwdLayout::kOffStage).
-bool encode_fwd_out(CUtensorMap* map, const void* o, int d, int N, int bh) {
+// Outputs stored from per-warp staging boxes (the forward's O, the backward's
+// dK and dV): 32 x 32 boxes (64-byte rows), 64-byte swizzle
+// (fa::FwdLayout::kOffStage, fa::BwdLayout::kOffStage).
+bool encode_out_box32(CUtensorMap* map, const void* o, int d, int N, int bh) {
   return encode_bf16_3d_box(map, o, d, N, bh, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
@@ -259,11 +260,16 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   }
   {
     LaunchTimer timer(st, FA_KERNEL_BWD_MAIN);
-    // one CTA per (head, key tile); the kernel maps the linear index to them
-    dim3 grid(static_cast<unsigned>(BH) * static_cast<unsigned>(np / 128));
+    // work items (head, key tile); persistent: one CTA per SM, the kernel
+    // maps item numbers to them
+    const long long items = static_cast<long long>(BH) * (np / 128);
+    if (items > 0x7fffffffLL) return FA_ERR_SHAPE;
+    const int n_items = static_cast<int>(items);
+    const int grid = std::min(n_items, sm_count(dev));
+    const uint32_t slot = next_sched_slot(dev);
     fa::bwd_main_kernel<D, C, !kDet><<<grid, L::kThreads, L::kSmemAlloc, st>>>(
         mq, mk, mv, mdo, mdk, mdv, ws.dvec, ws.lse2, ws.dq_acc, N, np, scale, c_exp,
-        kWaitLimitNs);
+        kWaitLimitNs, BH, n_items, slot);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (kDet) {
@@ -302,7 +308,7 @@ fa_status bwd_entry(const void* q, const void* k, const void* v, const void* o, 
   CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
   if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
       !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_bf16_3d(&mdo, dout, d, N, bh, 128) ||
-      !encode_bf16_3d(&mdk, dk, d, N, bh, 128) || !encode_bf16_3d(&mdv, dv, d, N, bh, 128) ||
+      !encode_out_box32(&mdk, dk, d, N, bh) || !encode_out_box32(&mdv, dv, d, N, bh) ||
       !encode_bf16_3d(&mdq, dq, d, N, bh, 128))
     return FA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -370,7 +376,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   const int bh = B * H;
   CUtensorMap mq, mk, mv, mo;
   if (!encode_bf16_3d(&mq, q, d, N, bh, 128) || !encode_bf16_3d(&mk, k, d, N, bh, 128) ||
-      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_fwd_out(&mo, o, d, N, bh))
+      !encode_bf16_3d(&mv, v, d, N, bh, 128) || !encode_out_box32(&mo, o, d, N, bh))
     return FA_ERR_CUDA;
   const float scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
