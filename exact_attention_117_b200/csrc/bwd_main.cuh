@@ -351,12 +351,14 @@ __global__ void __launch_bounds__(384, 1)
     constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);
     constexpr uint32_t id_kmn = idesc_bf16_f32(128, D, false, true);
     constexpr uint32_t id_mnmn = idesc_bf16_f32(128, D, true, true);
-    // With dQ the MMA loops stay rolled, which keeps the hot code of the MMA,
-    // compute and dQ warps that share a scheduler within its instruction
-    // cache (B200: no_instruction stalls down; B=64 H=16 N=1024 causal +18 %,
-    // B=16 H=16 N=4096 d=64 +15 %).  Without dQ the tensor pipe is the busier
-    // unit and unrolled issue measured faster (B=2 H=16 N=4096: +8 %).
-    constexpr int kMmaUnroll = kDq ? 1 : 8;
+    // With dQ the MMA loops are unrolled only by 2, which keeps the hot code
+    // of the MMA, compute and dQ warps that share a scheduler within its
+    // instruction cache (B200, against full unrolling: no_instruction stalls
+    // down, B=64 H=16 N=1024 causal +18 %, B=16 H=16 N=4096 d=64 +15 %;
+    // against no unrolling: B=2 H=16 N=4096 +2 %).  Without dQ the tensor
+    // pipe is the busier unit and full unrolling measured faster (B=2 H=16
+    // N=4096: +8 %).
+    constexpr int kMmaUnroll = kDq ? 2 : 8;
     const uint32_t err = err_k | kErrRoleMma;
     const uint32_t a_k = sb + L::kOffK, a_v = sb + L::kOffV, a_ds = sb + L::kOffDS;
     const uint64_t d_ones = sw32_slab_desc(sb + L::kOffOnes);
