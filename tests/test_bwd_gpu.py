@@ -124,6 +124,26 @@ def test_bwd_poisoned_outputs_fully_written():
         assert torch.isfinite(t.float()).all()
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("deterministic", [False, True])
+def test_bwd_many_items_per_cta(d, deterministic):
+    # 4 x 40 heads x 5 key tiles = 800 (head, key tile) work items for the
+    # persistent main kernel, several per CTA and of 1 to 5 query tiles each
+    # under the causal mask (N = 600: the last key tile is ragged).  Every
+    # output element must be written, and the first head, one in the middle
+    # and the last (whose items are claimed last) must match the oracle.
+    w = Workload("items", 4, 40, 600, d, seed_base=53)
+    x = make_inputs(w, DEV)
+    o, lse = fa.forward(x["q"], x["k"], x["v"], causal=True)
+    dq, dk, dv = (torch.full_like(x["q"], float("nan")) for _ in range(3))
+    fa.backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal=True, dq=dq, dk=dk, dv=dv,
+                deterministic=deterministic)
+    fa.check_device_error()
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+    _check(x, (dq, dk, dv), True, w.scale, [(0, 0), (2, 17), (3, 39)])
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.09])
 @pytest.mark.parametrize("causal", [False, True])
 def test_bwd_any_finite_scale(scale, causal):
