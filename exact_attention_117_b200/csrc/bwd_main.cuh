@@ -148,24 +148,24 @@ __device__ __forceinline__ void split3(float x, float& a, float& b, float& c) {
 
 // kDq = false (deterministic backward): no dQ MMA and no atomics here; dQ
 // comes from dq_pass_kernel.  dP_{i+1} then only waits for dS_i to be formed.
-constexpr int kHeadGroup = 8;
 // pause after each pair of dQ vector adds (d = 128)
 constexpr uint32_t kAddGapNs = 80;
 
-// Work item `lin` -> (head, key tile).  Items run in groups of kHeadGroup
-// heads, and within a group key tile 0 of every head first, then key tile 1,
-// ... (small j = the longest loop under the causal mask).  The CTAs busy at
-// any time then share the Q, dO and dQ accumulator tiles of a few heads,
-// which stay in L2, and the last items of a launch are short ones.
+// Work item `lin` -> (head, key tile).  Items run in groups of `hg` heads
+// (chosen by the host from the heads' L2 footprint), and within a group key
+// tile 0 of every head first, then key tile 1, ... (small j = the longest
+// loop under the causal mask).  The CTAs busy at any time then share the Q,
+// dO and dQ accumulator tiles of a few heads, which stay in L2, and the last
+// items of a launch are short ones.
 struct BwdItem {
   int bh, j, i0, n_it;
 };
 template <bool kCausal>
-__device__ __forceinline__ BwdItem bwd_item(int lin, int n_kt, int bh_count) {
-  const int grp = lin / (kHeadGroup * n_kt);
-  const int g_base = grp * kHeadGroup;
-  const int g_size = min(kHeadGroup, bh_count - g_base);
-  const int g_off = lin - grp * kHeadGroup * n_kt;
+__device__ __forceinline__ BwdItem bwd_item(int lin, int n_kt, int bh_count, int hg) {
+  const int grp = lin / (hg * n_kt);
+  const int g_base = grp * hg;
+  const int g_size = min(hg, bh_count - g_base);
+  const int g_off = lin - grp * hg * n_kt;
   BwdItem w;
   w.bh = g_base + g_off % g_size;
   w.j = g_off / g_size;
@@ -181,7 +181,8 @@ __global__ void __launch_bounds__(384, 1)
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                     const float* __restrict__ dvec, const float* __restrict__ lse2,
                     float* __restrict__ dq_acc, int n, int np, float scale, float c_exp,
-                    uint64_t limit_ns, int bh_count, int n_items, uint32_t sched_slot) {
+                    uint64_t limit_ns, int bh_count, int n_items, uint32_t sched_slot,
+                    int head_group) {
   using L = BwdLayout<D>;
   constexpr int kDBlk = D / 64;
   constexpr int DS = L::kDoStages;
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(384, 1)
     int item = static_cast<int>(blockIdx.x);
     for (int k = 0; publish(k, item); ++k) {
       if (item < 0) break;
-      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count);
+      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count, head_group);
       bool ok = true;
       if (lane == 0) {
         // a failed check raises the abort flag; the other roles then give up
@@ -328,7 +329,7 @@ __global__ void __launch_bounds__(384, 1)
       item = f >= static_cast<unsigned int>(n_items) - gridDim.x ? -1
                                                                   : static_cast<int>(gridDim.x + f);
       if (lane == 0 && item >= 0) {
-        const BwdItem nw = bwd_item<kCausal>(item, n_kt, bh_count);
+        const BwdItem nw = bwd_item<kCausal>(item, n_kt, bh_count, head_group);
         for (int db = 0; db < kDBlk; ++db) {
           tma_prefetch_l2_3d(&tm_k, db * 64, nw.j * 128, nw.bh);
           tma_prefetch_l2_3d(&tm_v, db * 64, nw.j * 128, nw.bh);
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int k = 0;; ++k) {
       int item = -1;
       if (!read_item(k, item, err) || item < 0) break;
-      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count);
+      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count, head_group);
       // the first dP overwrites the columns of the previous item's last dQ
       bool ok = wait_bounded_warp(bar(L::kKvFull), k & 1, limit_ns, abort_flag, err) &&
                 wait_bounded_warp(bar(L::kQFull + (gq & 1)), (gq >> 1) & 1, limit_ns, abort_flag,
@@ -503,7 +504,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int k = 0; ok; ++k) {
       int item = -1;
       if (!read_item(k, item, err) || item < 0) break;
-      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count);
+      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count, head_group);
       for (int it = 0; it < w.n_it; ++it) {
         const int t = gq + it;
         const int i = w.i0 + it;
@@ -572,7 +573,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int k = 0; ok; ++k) {
       int item = -1;
       if (!read_item(k, item, err) || item < 0) break;
-      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count);
+      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count, head_group);
       const bool key_ok = w.j * 128 + r < n;
       for (int it = 0; it < w.n_it; ++it) {
         const int t = gq + it;
@@ -741,7 +742,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int k = 0; ok; ++k) {
       int item = -1;
       if (!read_item(k, item, err) || item < 0) break;
-      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count);
+      const BwdItem w = bwd_item<kCausal>(item, n_kt, bh_count, head_group);
       for (int it = 0; it < w.n_it; ++it) {
         const int t = gq + it;
         const int i = w.i0 + it;

@@ -125,8 +125,8 @@ fa_status check_common(int B, int H, int N, int d, float scale) {
   if (bh > 0x7fffffffLL) return FA_ERR_SHAPE;
   // kernels that put 128-row tiles on grid.y (the dQ pass) need at most 65535
   if (N > (65535 * 128)) return FA_ERR_SHAPE;
-  // the backward main kernel runs a linear grid of B*H*ceil(N/128) CTAs, and
-  // the kernels index blocks with 32-bit signed arithmetic
+  // the backward main kernel numbers its B*H*ceil(N/128) work items, and the
+  // kernels index blocks and items with 32-bit signed arithmetic
   if (bh * ((static_cast<long long>(N) + 127) / 128) > 0x7fffffffLL) return FA_ERR_SHAPE;
   if (static_cast<long long>(N) * bh > (1LL << 40)) return FA_ERR_SHAPE;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED_D;
@@ -221,6 +221,20 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Heads per launch-order group of the backward main kernel.  The busy CTAs
+// share the Q, dO and fp32 dQ accumulator tiles of a group through L2, 8 N d
+// bytes per head; groups of about kBwdGroupBytes, 4 to 64 heads, measured
+// best among 32, 64 and 128 MB and a fixed 8 heads (B200, causal, atomic
+// backward main kernel, 64 MB against 8 heads: B=64 H=16 N=512 560 vs 502
+// TFLOP/s, B=16 H=16 N=4096 d=64 667 vs 591, B=1 H=32 N=16384 1023 vs 981,
+// B=2 H=16 N=4096 981 vs 968; the deterministic one unchanged).
+constexpr long long kBwdGroupBytes = 64LL << 20;
+int bwd_head_group(int BH, int np, int d) {
+  const long long per_head = 8LL * np * d;
+  const long long g = std::max(4LL, std::min(64LL, kBwdGroupBytes / per_head));
+  return static_cast<int>(std::min<long long>(g, BH));
+}
+
 template <int D, bool C, bool kDet>
 fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
@@ -269,7 +283,7 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
     const uint32_t slot = next_sched_slot(dev);
     fa::bwd_main_kernel<D, C, !kDet><<<grid, L::kThreads, L::kSmemAlloc, st>>>(
         mq, mk, mv, mdo, mdk, mdv, ws.dvec, ws.lse2, ws.dq_acc, N, np, scale, c_exp,
-        kWaitLimitNs, BH, n_items, slot);
+        kWaitLimitNs, BH, n_items, slot, bwd_head_group(BH, np, D));
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (kDet) {
