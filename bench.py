@@ -57,8 +57,13 @@ def rank_workload(w, rank):
     return dataclasses.replace(w, seed_base=w.seed_base + 1000 * rank)
 
 
-# groups of (b, h) slices in the end-to-end leg (copies overlap compute)
-E2E_CHUNKS = 4
+# groups of (b, h) slices in the end-to-end leg (copies overlap compute).  The
+# copies bound it (B200, PCIe: 55 GB/s one way, 50 GB/s each way at once, so
+# 2.7 ms of copies per c3 step); B200, c3: 1 group 3.42 ms per step, 2 groups
+# 2.95, 3 groups 3.26, 4 groups 3.13, 16 groups 3.67 -- more groups overlap
+# more, but each call on fewer heads fills the GPU less (8 heads: 128 forward
+# items for 148 SMs).
+E2E_CHUNKS = 2
 
 
 def max_over_ranks(values, world, device=None):
@@ -466,7 +471,7 @@ def run_ours(args, w, rank, world, local_rank):
         # them: its copy-in waits for that step's compute of the group, its
         # compute for that step's copy-out.
         bh = w.B * w.H
-        n_chunks = max(1, min(E2E_CHUNKS, bh))
+        n_chunks = max(1, min(args.e2e_chunks, bh))
         bounds = [(c * bh // n_chunks, (c + 1) * bh // n_chunks) for c in range(n_chunks)]
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         s_comp = stream
@@ -978,6 +983,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c3", choices=["c3", "c4"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=E2E_CHUNKS,
+                    help="groups of (b, h) slices the end-to-end leg pipelines its copies over")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-long-context", action="store_true",
                     help="skip the long-context (B=1 H=32 N=16384) leg of the default line")
