@@ -199,16 +199,16 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   }
   const int q_tiles = (N + L::kBM - 1) / L::kBM;
   const int pairs = (q_tiles + 1) / 2;
-  // Work items: (head, pair of Q tiles[, split]).  Up to 48 heads form one
-  // launch-order group; more heads go in groups whose K and V (4 N d bytes
-  // per head) come to about 32 MB, 8 to 128 heads, which the busy CTAs share
-  // in L2 (B200, causal, B*H*N = 2^20, against a fixed 32 heads: N = 512
-  // d = 128 128 heads 505 vs 468 TFLOP/s, N = 8192 8 heads 1172 vs 1124;
-  // within 2 % of the best group size at N = 1024 / 2048 and d = 64).
+  // Work items: (head, pair of Q tiles[, split]).  The heads go in
+  // launch-order groups whose K and V (4 N d bytes per head) come to about
+  // 32 MB, 8 to 128 heads (fewer if there are fewer), which the busy CTAs
+  // share in L2 (B200, causal, against a fixed 32 heads: B*H*N = 2^20 at
+  // N = 512 d = 128 128 heads 505 vs 468 TFLOP/s, N = 8192 8 heads 1172 vs
+  // 1124; B=1 H=32 N=16384 8 heads 1234 vs 1176; B=2 H=16 N=4096 16 heads
+  // as fast as 32; within 2 % of the best size at N = 1024 / 2048, d = 64).
   const long long kv_bytes = 4LL * q_tiles * L::kBM * D;
   const int head_group =
-      BH <= 48 ? BH
-               : static_cast<int>(std::max(8LL, std::min(128LL, (32LL << 20) / kv_bytes)));
+      static_cast<int>(std::max(8LL, std::min(128LL, (32LL << 20) / kv_bytes)));
   const long long items = static_cast<long long>(BH) * pairs * (kSplit ? num_splits : 1);
   if (items > 0x7fffffffLL) return FA_ERR_SHAPE;
   const int n_items = static_cast<int>(items);
