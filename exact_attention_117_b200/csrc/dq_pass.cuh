@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(384, 1)
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ dvec,
                    const float* __restrict__ lse2, int n, int np, float scale, float c_exp,
-                   uint64_t limit_ns) {
+                   uint64_t limit_ns, int bh_count, int head_group) {
   using L = DqLayout<D>;
   constexpr int KS = L::kKStages;
   constexpr int VS = L::kVStages;
@@ -83,9 +83,18 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
+  // Launch order: heads in groups of head_group, and within a group the
+  // longest causal rows first (Q tile n-1 of every head of the group, then
+  // n-2, ...), so the CTAs in flight share the K and V tiles of a few heads
+  // in L2.
   const int n_tiles = np / 128;
-  const int i = n_tiles - 1 - static_cast<int>(blockIdx.y);  // longest causal rows first
+  const int lin = static_cast<int>(blockIdx.x);
+  const int grp = lin / (head_group * n_tiles);
+  const int g_base = grp * head_group;
+  const int g_size = min(head_group, bh_count - g_base);
+  const int g_off = lin - grp * head_group * n_tiles;
+  const int bh = g_base + g_off % g_size;
+  const int i = n_tiles - 1 - g_off / g_size;
   const int n_kv = kCausal ? i + 1 : n_tiles;
   const unsigned int err_k = kErrBwdDq;
 

@@ -123,7 +123,8 @@ fa_status check_common(int B, int H, int N, int d, float scale) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > 0x7fffffffLL) return FA_ERR_SHAPE;
-  // kernels that put 128-row tiles on grid.y (the dQ pass) need at most 65535
+  // sequence length bound (8.4 M rows), far beyond what fits in device memory
+  // at any B*H: row and tile indices stay well inside 32-bit arithmetic
   if (N > (65535 * 128)) return FA_ERR_SHAPE;
   // the backward main kernel numbers its B*H*ceil(N/128) work items, and the
   // kernels index blocks and items with 32-bit signed arithmetic
@@ -294,9 +295,14 @@ fa_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   }
   if (kDet) {
     LaunchTimer timer(st, FA_KERNEL_BWD_DQ);
-    dim3 grid(static_cast<unsigned>(BH), static_cast<unsigned>(np / 128));
+    // one CTA per (head, Q tile), numbered in head groups whose K and V come
+    // to about 32 MB, as the forward's
+    const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(np / 128);
+    const long long kv_bytes = 4LL * np * D;
+    const int hg = static_cast<int>(std::max(8LL, std::min(128LL, (32LL << 20) / kv_bytes)));
     fa::dq_pass_kernel<D, C><<<grid, LQ::kThreads, LQ::kSmemAlloc, st>>>(
-        mq, mk, mv, mdo, mdq, ws.dvec, ws.lse2, N, np, scale, scale_log2, kWaitLimitNs);
+        mq, mk, mv, mdo, mdq, ws.dvec, ws.lse2, N, np, scale, scale_log2, kWaitLimitNs, BH,
+        std::min(hg, BH));
   } else {
     LaunchTimer timer(st, FA_KERNEL_BWD_DQ);
     const long long warps = (static_cast<long long>(BH) * N + 15) / 16 * (D / 16);

@@ -73,7 +73,7 @@ def test_shapes_beyond_the_grid_limits(lib):
     # B*H and N are each within their own limits
     assert _fwd(lib, B=1 << 20, H=1, N=1 << 18) == 2
     assert _bwd(lib, B=1 << 20, H=1, N=1 << 18, ws_bytes=1 << 62) == 2
-    # 128-row tiles on grid.y: N up to 65535 * 128
+    # the sequence-length bound: N up to 65535 * 128
     assert _fwd(lib, N=65535 * 128 + 1) == 2
 
 
