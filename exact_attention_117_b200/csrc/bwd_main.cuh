@@ -43,8 +43,8 @@
 // dK_j and dV_j accumulate in TMEM and are written once per item (no
 // atomics): each compute warp converts its 32 key rows to bf16 through two
 // 32 x 32 staging boxes (64-byte swizzle) that one lane stores with TMA.  dQ_i
-// partial products are read out of TMEM by a separate warp group and added
-// into the fp32 accumulator with vector atomic adds.  The accumulator keeps
+// partial products are read out of TMEM (by a separate warp group at d = 128)
+// and added into the fp32 accumulator with vector atomic adds.  The accumulator keeps
 // each 128-row tile as [D/4 column groups][128 rows][4 floats] so that those
 // adds are coalesced.  For d = 128 the 64 KB of adds of one Q tile are paced,
 // an 80 ns sleep after each pair of vector adds (about 1.3 us in all, under
@@ -57,15 +57,22 @@
 //
 // Warp roles (384 threads): warp 0 TMA producer and scheduler; warp 1 TMEM
 // allocator and MMA issuer; warp 2 builds the LSE / D slabs; warps 4-7
-// compute P^T / dS^T (thread = key row) and write dK, dV; warps 8-11 read dQ
-// out of TMEM (thread = query row) and add it to global.  Without dQ (the
-// deterministic backward) warps 8-11 instead share the P^T / dS^T work: each
-// warp group takes 64 of the 128 query columns (and the same half of dK, dV).
+// compute P^T / dS^T (thread = key row) and write dK, dV; at d = 128 warps
+// 8-11 read dQ out of TMEM (thread = query row) and add it to global.
+// Without dQ (the deterministic backward), and with dQ at d = 64, warps 8-11
+// instead share the P^T / dS^T work: each warp group takes 64 of the 128
+// query columns (and the same half of the columns of dK, dV and dQ, whose
+// read-out the two groups then do between a tile's P^T and its dS^T).  At
+// d = 128 dQ reuses dP'^T's TMEM columns, so the next dP waits for its
+// read-out, which only a warp group of its own does at once (the compute
+// warps doing it: B=2 H=16 N=4096 -8 %); at d = 64 dQ has columns of its own
+// and the shared work pays (B=16 H=16 N=4096 +11 %, N=1024 +16 %).
 // P^T of query half h sits in the first 32 of the 64 TMEM columns S'^T had
 // for those queries.
 //
 // TMEM columns:  dK [0,D), dV [D,2D), S'^T/P^T [2D,2D+128), dP'^T [2D+128,2D+256);
-// dQ reuses the dP'^T columns once dS^T has been formed (d=128 fills all 512).
+// at d = 128 dQ reuses the dP'^T columns once dS^T has been formed (all 512
+// are taken), at d = 64 it has [384, 448).
 #pragma once
 
 namespace fa {
@@ -112,8 +119,11 @@ struct BwdLayout {
   static constexpr uint32_t kColDV = D;
   static constexpr uint32_t kColS = 2 * D;
   static constexpr uint32_t kColDP = 2 * D + 128;
-  static constexpr uint32_t kColDQ = kColDP;
-  static_assert(kColDP + 128 <= kTmemCols, "TMEM budget");
+  // d = 128 fills all 512 columns, so dQ reuses dP'^T's once dS^T is formed;
+  // at d = 64 it has columns of its own
+  static constexpr bool kDqOwnCols = (D == 64);
+  static constexpr uint32_t kColDQ = kDqOwnCols ? kColDP + 128 : kColDP;
+  static_assert(kColDP + 128 <= kTmemCols && kColDQ + D <= kTmemCols, "TMEM budget");
 };
 
 // Shared-memory descriptor of a 128 x 16 bf16 K-major slab with 32-byte
@@ -186,6 +196,13 @@ __global__ void __launch_bounds__(384, 1)
   using L = BwdLayout<D>;
   constexpr int kDBlk = D / 64;
   constexpr int DS = L::kDoStages;
+  // With dQ at d = 64 (own TMEM columns) all eight compute warps share the
+  // P^T / dS^T work by query halves and read dQ out themselves; at d = 128
+  // warps 4-7 compute and warps 8-11 read dQ out (its columns are dP'^T's,
+  // so the next dP waits for the read-out, which a separate warp group does
+  // at once).
+  constexpr bool kSplitDq = kDq && L::kDqOwnCols;
+  constexpr bool kEight = !kDq || kSplitDq;  // eight compute warps
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -206,7 +223,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t cnt = 1;
       if (b == L::kDqFree) cnt = 4;  // the dQ read-out warps
       if (b == L::kPReady || b == L::kDsReady || b == L::kDkdvFree)
-        cnt = kDq ? 4 : 8;  // the compute warps
+        cnt = kEight ? 8 : 4;  // the compute warps
       if ((b >= L::kQFull && b < L::kQFull + 2) || (b >= L::kDoFull && b < L::kDoFull + 2))
         cnt = 2;  // the TMA producer and the slab builder
       if (b == L::kItemEmpty || b == L::kItemEmpty + 1) cnt = L::kItemReaders;
@@ -359,7 +376,7 @@ __global__ void __launch_bounds__(384, 1)
     // against no unrolling: B=2 H=16 N=4096 +2 %).  Without dQ the tensor
     // pipe is the busier unit and full unrolling measured faster (B=2 H=16
     // N=4096: +8 %).
-    constexpr int kMmaUnroll = kDq ? 2 : 8;
+    constexpr int kMmaUnroll = (kDq && !kSplitDq) ? 2 : 8;
     const uint32_t err = err_k | kErrRoleMma;
     const uint32_t a_k = sb + L::kOffK, a_v = sb + L::kOffV, a_ds = sb + L::kOffDS;
     const uint64_t d_ones = sw32_slab_desc(sb + L::kOffOnes);
@@ -399,7 +416,7 @@ __global__ void __launch_bounds__(384, 1)
                                   err) &&
                 wait_bounded_warp(bar(L::kDoFull + gq % DS), (gq / DS) & 1, limit_ns, abort_flag,
                                   err) &&
-                (!kDq || gq == 0 ||
+                (!kDq || kSplitDq || gq == 0 ||
                  wait_bounded_warp(bar(L::kDqFree), (gq - 1) & 1, limit_ns, abort_flag, err));
       if (!ok) break;
       tc_fence_after();
@@ -470,7 +487,8 @@ __global__ void __launch_bounds__(384, 1)
         tc_commit(bar(L::kQEmpty + st));  // Q_i and its slab are no longer read
         tc_commit(bar(L::kDsFree));
         if (next) {  // dP of the next Q tile once dQ_i has left the shared columns
-          if (kDq && !wait_bounded_warp(bar(L::kDqFree), ph, limit_ns, abort_flag, err)) {
+          if (kDq && !kSplitDq &&
+              !wait_bounded_warp(bar(L::kDqFree), ph, limit_ns, abort_flag, err)) {
             ok = false;
             break;
           }
@@ -552,13 +570,14 @@ __global__ void __launch_bounds__(384, 1)
       }
       gq += w.n_it;
     }
-  } else if (warp >= 4 && (warp < 8 || !kDq)) {
+  } else if (warp >= 4 && (warp < 8 || kEight)) {
     // ------------------------------------------------ P^T, dS^T, dK / dV out
-    // kDq: warps 4-7 take all 128 query columns; otherwise warps 4-7 take
-    // queries 0-63 and warps 8-11 queries 64-127 (and the two halves of dK, dV)
-    constexpr int kHalves = kDq ? 2 : 1;
-    constexpr int kBoxes = kDq ? 2 : 1;  // staging boxes of this warp
-    const int h0 = kDq ? 0 : (warp >> 2) - 1;
+    // four compute warps: warps 4-7 take all 128 query columns; eight: warps
+    // 4-7 take queries 0-63 and warps 8-11 queries 64-127 (and the two halves
+    // of the columns of dK, dV and, with dQ, dQ)
+    constexpr int kHalves = kEight ? 1 : 2;
+    constexpr int kBoxes = kEight ? 1 : 2;  // staging boxes of this warp
+    const int h0 = kEight ? (warp >> 2) - 1 : 0;
     const int r = (warp & 3) * 32 + lane;  // key row in the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t err = err_k | kErrRoleSoftmax;
@@ -568,6 +587,31 @@ __global__ void __launch_bounds__(384, 1)
                             tmem_range_ok(tmem + lane_off + L::kColDV, tmem, D, L::kTmemCols) &&
                             tmem_range_ok(tmem + lane_off + L::kColS, tmem, 128, L::kTmemCols),
                         err, abort_flag);
+    // (eight compute warps with dQ) dQ of Q tile i, tile t of this CTA's
+    // sequence: once its MMA is done this warp group reads its half of the
+    // columns for the 128 query rows (thread = query row = TMEM lane) and adds
+    // them into the fp32 accumulator, laid out as for the read-out warps below
+    auto dq_out = [&](int t, int i, int bh) -> bool {
+      if (!wait_bounded_warp(bar(L::kDqFull), t & 1, limit_ns, abort_flag, err_k | kErrRoleDq))
+        return false;
+      tc_fence_after();
+      uint32_t u[D / 2];
+#pragma unroll
+      for (int cc = 0; cc < D / 64; ++cc)
+        tmem_ld_32x32b_x32(tmem + lane_off + L::kColDQ + h0 * (D / 2) + cc * 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(&u[cc * 32]));
+      tmem_wait_ld_regs(u);
+      if (!dbg_check(static_cast<size_t>(bh) * n_kt + i < static_cast<size_t>(bh_count) * n_kt,
+                     err_k | kErrRoleDq, abort_flag))
+        return false;
+      float* dst = dq_acc + (static_cast<size_t>(bh) * n_kt + static_cast<size_t>(i)) * 128 * D +
+                   static_cast<size_t>(h0) * (D / 8) * 512 + static_cast<size_t>(r) * 4;
+#pragma unroll
+      for (int q = 0; q < D / 8; ++q)
+        red_add_v4(dst + q * 512, __uint_as_float(u[4 * q]), __uint_as_float(u[4 * q + 1]),
+                   __uint_as_float(u[4 * q + 2]), __uint_as_float(u[4 * q + 3]));
+      return true;
+    };
     int gq = 0;
     int n_box = 0;  // staging boxes this warp has filled
     for (int k = 0; ok; ++k) {
@@ -623,6 +667,13 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::kPReady));
+        // dQ of the previous Q tile, while this tile's dV and the previous
+        // tile's dK run on the tensor core (the next dQ MMA waits for this
+        // tile's dS, which these warps form after the read-out)
+        if (kSplitDq && it > 0 && !dq_out(t - 1, i - 1, w.bh)) {
+          ok = false;
+          break;
+        }
 
         // with dQ, dS^T goes to shared memory (dK and dQ read it there) once the
         // previous tile's MMAs are done with it; without dQ it goes over the
@@ -666,6 +717,10 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) mbar_arrive(bar(L::kDsReady));
       }
       if (!ok) break;
+      if (kSplitDq && !dq_out(gq + w.n_it - 1, w.i0 + w.n_it - 1, w.bh)) {
+        ok = false;
+        break;
+      }
       gq += w.n_it;
       // ----------------------------------------------------- dK, dV epilogue
       // Once the item's MMAs are done: per 32 columns each thread converts
@@ -681,8 +736,8 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       tc_fence_after();
-      constexpr int kCols = D / 32 / (kDq ? 1 : 2);  // 32-column boxes per matrix
-      const int c_first = kDq ? 0 : h0 * kCols;
+      constexpr int kCols = D / 32 / (kEight ? 2 : 1);  // 32-column boxes per matrix
+      const int c_first = kEight ? h0 * kCols : 0;
       const int row0 = w.j * 128 + (warp & 3) * 32;  // first key row of this warp's boxes
       // (loops kept rolled: this code runs once per item, and unrolled it
       // would crowd the hot loops out of the instruction cache)
@@ -732,7 +787,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     // the staging boxes must be read out before the CTA's shared memory goes
     if (lane == 0) bulk_wait_group_read_0();
-  } else if (kDq && warp >= 8) {
+  } else if (kDq && !kSplitDq && warp >= 8) {
     // --------------------------------------------------------- dQ read-out
     const int c = threadIdx.x - 256;  // query row in the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
