@@ -144,6 +144,10 @@ def _clock_worker(index, conn, period_s):
     get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
         pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
     mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+    # one query of each kind before the region: the first calls are slow (a
+    # 12 ms region once got no sample of its own)
+    pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    get(h)
     out = []
     conn.send("ready")
     while not conn.poll():
