@@ -37,16 +37,17 @@
 // and the compute warps store the current item's dK_j, dV_j while the next
 // item's first scores are computed.  With one CTA per item, a CTA's fixed
 // costs (set-up, first loads, pipeline fill and drain, epilogue) were paid
-// once per key tile, which dominated short sequences (B=64 H=32 N=512 causal:
+// once per key tile, which dominated short sequences (B=128 H=16 N=512 causal:
 // about 17k cycles per CTA against 5.6k per Q tile).
 //
 // dK_j and dV_j accumulate in TMEM and are written once per item (no
-// atomics): each compute warp converts its 32 key rows to bf16 through two
-// 32 x 32 staging boxes (64-byte swizzle) that one lane stores with TMA.  dQ_i
-// partial products are read out of TMEM (by a separate warp group at d = 128)
-// and added into the fp32 accumulator with vector atomic adds.  The accumulator keeps
-// each 128-row tile as [D/4 column groups][128 rows][4 floats] so that those
-// adds are coalesced.  For d = 128 the 64 KB of adds of one Q tile are paced,
+// atomics): each compute warp converts its 32 key rows to bf16 through
+// 32 x 32 staging boxes (64-byte swizzle; two per warp with four compute
+// warps, one with eight) that one lane stores with TMA.  dQ_i partial
+// products are read out of TMEM (by a separate warp group at d = 128) and
+// added into the fp32 accumulator with vector atomic adds.  The accumulator
+// keeps each 128-row tile as [D/4 column groups][128 rows][4 floats] so that
+// those adds are coalesced.  For d = 128 the 64 KB of adds of one Q tile are paced,
 // an 80 ns sleep after each pair of vector adds (about 1.3 us in all, under
 // half of a Q-loop iteration): issued as one burst they queue ahead of the
 // next tile loads and stretch every iteration (B200: 857 -> 940 TFLOP/s for
@@ -66,7 +67,7 @@
 // d = 128 dQ reuses dP'^T's TMEM columns, so the next dP waits for its
 // read-out, which only a warp group of its own does at once (the compute
 // warps doing it: B=2 H=16 N=4096 -8 %); at d = 64 dQ has columns of its own
-// and the shared work pays (B=16 H=16 N=4096 +11 %, N=1024 +16 %).
+// and the shared work pays (B=16 H=16 N=4096 +11 %, B=64 H=16 N=1024 +16 %).
 // P^T of query half h sits in the first 32 of the 64 TMEM columns S'^T had
 // for those queries.
 //

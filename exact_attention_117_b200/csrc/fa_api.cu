@@ -232,7 +232,7 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 // share the Q, dO and fp32 dQ accumulator tiles of a group through L2, 8 N d
 // bytes per head; groups of about kBwdGroupBytes, 4 to 64 heads, measured
 // best among 32, 64 and 128 MB and a fixed 8 heads (B200, causal, atomic
-// backward main kernel, 64 MB against 8 heads: B=64 H=16 N=512 560 vs 502
+// backward main kernel, 64 MB against 8 heads: B=128 H=16 N=512 560 vs 502
 // TFLOP/s, B=16 H=16 N=4096 d=64 667 vs 591, B=1 H=32 N=16384 1023 vs 981,
 // B=2 H=16 N=4096 981 vs 968; the deterministic one unchanged).
 constexpr long long kBwdGroupBytes = 64LL << 20;
